@@ -1,0 +1,119 @@
+"""Pins for the oracle's NVFP4 block quantiser and storage layouts (CPU only)."""
+import numpy as np
+import pytest
+
+from oracle import nvfp4_oracle as o
+import workloads as wk
+
+
+def _rand(rows, cols, seed=0, outliers=0):
+    return wk.activations(rows, cols, outliers, seed).float().numpy()
+
+
+def test_global_scale_puts_largest_block_scale_on_448():
+    x = _rand(64, 256, outliers=2)
+    q, s, G = o.quantize(x)
+    assert G == np.float32(np.max(np.abs(x)) / np.float32(2688))
+    assert s.max() == 0x7E                       # 448
+    # the block holding the tensor's amax uses the top scale
+    r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert s[r, c // 16] == 0x7E
+    # and its amax element maps to the top level (magnitude code 7, value 6)
+    assert q[r, c] & 7 == 7
+
+
+def test_idempotent_on_dequantised_values():
+    x = _rand(128, 512, seed=3, outliers=4)
+    q, s, G = o.quantize(x)
+    deq = o.dequantize(q, s, G).astype(np.float32)
+    q2, s2, G2 = o.quantize(deq, G)
+    assert np.array_equal(q2 & 7, q & 7)          # magnitudes
+    nz = (q & 7) != 0
+    assert np.array_equal(q2[nz], q[nz])          # signs where nonzero
+    assert np.array_equal(s2, s)
+
+
+def test_per_element_error_is_within_half_a_level_step():
+    x = _rand(64, 1024, seed=5, outliers=3)
+    q, s, G = o.quantize(x)
+    d = (o.e4m3_decode(s).astype(np.float32) * G).astype(np.float64)
+    dd = np.repeat(d, 16, axis=1)
+    t = np.abs(x.astype(np.float64)) / dd          # magnitude in level units
+    half = np.where(t < 2, 0.25, np.where(t < 4, 0.5, 1.0))
+    err = np.abs(np.abs(o.e2m1_decode(q)) - t)
+    sat = t > 6
+    assert np.all(err[~sat] <= half[~sat] * (1 + 1e-6))
+    assert np.all(q[sat] & 7 == 7)
+
+
+def test_zero_blocks_and_zero_tensor():
+    x = _rand(4, 64, seed=1)
+    x[1, 16:32] = 0
+    q, s, G = o.quantize(x)
+    assert s[1, 1] == 0 and np.all(q[1, 16:32] == 0)
+    q0, s0, G0 = o.quantize(np.zeros((4, 64), np.float32))
+    assert G0 == 0 and not q0.any() and not s0.any()
+
+
+def test_static_scale_saturates_instead_of_overflowing():
+    x = _rand(4, 64, seed=2)
+    G = np.float32(np.max(np.abs(x)) / 2688 / 8)   # 8x too small
+    q, s, _ = o.quantize(x, G)
+    assert s.max() == 0x7E
+    assert np.all(np.isfinite(o.dequantize(q, s, G)))
+
+
+def test_row_permutation_commutes_with_quantisation():
+    w = wk.weights(64, 256, 0.05, seed=4).float().numpy()
+    q, s, G = o.quantize(w)
+    qi, si, Gi = o.quantize(o.interleave_gate_up(w))
+    assert G == Gi
+    assert np.array_equal(qi, o.interleave_gate_up(q))
+    assert np.array_equal(si, o.interleave_gate_up(s))
+
+
+def test_dequantised_error_is_fp4_sized():
+    x = _rand(256, 1024, seed=6)
+    q, s, G = o.quantize(x)
+    deq = o.dequantize(q, s, G)
+    rel = np.linalg.norm(deq - x) / np.linalg.norm(x)
+    assert 0.05 < rel < 0.15
+
+
+def test_interleave_is_a_bijection_pairing_gate_and_up():
+    nh = 8
+    rows = np.arange(2 * nh)
+    p = o.interleave_gate_up(rows)
+    assert sorted(p.tolist()) == rows.tolist()
+    assert np.array_equal(p[0::2], np.arange(nh))
+    assert np.array_equal(p[1::2], np.arange(nh) + nh)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 64), (256, 512), (130, 80), (1, 16)])
+def test_scale_layout_is_a_bijection_onto_the_buffer(rows, cols):
+    nkb = cols // 16
+    rp = ((rows + 127) // 128) * 128
+    kp = ((nkb + 3) // 4) * 4
+    rr, kk = np.meshgrid(np.arange(rp), np.arange(kp), indexing="ij")
+    off = o.sf_offset(rr, kk, cols)
+    assert off.min() == 0 and off.max() == o.sf_bytes(rows, cols) - 1
+    assert len(np.unique(off)) == off.size
+    # every 128-row x 4-block unit is one contiguous 512-byte range
+    for r0 in range(0, rp, 128):
+        for k0 in range(0, kp, 4):
+            u = off[r0:r0 + 128, k0:k0 + 4]
+            assert u.max() - u.min() == 511 and u.min() % 512 == 0
+    # within a unit, 32 consecutive rows are 16 bytes apart (one line each)
+    assert np.all(np.diff(off[:32, 0]) == 16)
+
+
+def test_scale_and_code_packing_roundtrip():
+    rng = np.random.default_rng(0)
+    s = rng.integers(0, 0x7F, size=(200, 12), dtype=np.uint8)
+    buf = o.pack_scales(s, 192)
+    assert np.array_equal(o.unpack_scales(buf, 200, 192), s)
+    c = rng.integers(0, 16, size=(5, 64), dtype=np.uint8)
+    p = o.pack_codes(c)
+    assert p.shape == (5, 32)
+    assert np.array_equal(p[:, 0] & 0xF, c[:, 0]) and np.array_equal(p[:, 0] >> 4, c[:, 1])
+    assert np.array_equal(o.unpack_codes(p), c)
