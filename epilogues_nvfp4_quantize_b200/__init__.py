@@ -1,0 +1,22 @@
+"""NVFP4 block-scaled GEMM with fused RMSNorm / SwiGLU (+ NVFP4 re-quantisation)
+epilogues for B200 (sm_100a), exposed through the C ABI of libnvfp4epi.so.
+
+The Python names mirror the C entry points of include/nvfp4epi.h.
+"""
+from ._lib import (  # noqa: F401
+    EXPORTS,
+    LIB_PATH,
+    NVFP4Tensor,
+    gemm_nvfp4_plain,
+    gemm_nvfp4_rmsnorm,
+    gemm_nvfp4_swiglu,
+    launch_count,
+    load,
+    nvfp4_quantize,
+    quantize_workspace_bytes,
+    read_device_status,
+    rmsnorm_heads_bf16,
+    selftest_bounded_wait,
+    sf_bytes,
+    swiglu_bf16,
+)

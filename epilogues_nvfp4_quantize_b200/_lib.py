@@ -1,0 +1,182 @@
+"""ctypes binding of libnvfp4epi.so: argument marshalling only.
+
+Every computation runs in the library's CUDA kernels; this module turns torch tensors
+into device pointers, sizes and the current stream, and raises RuntimeError on a
+non-OK status. There is no CPU fallback: if the shared library is missing or cannot
+be loaded, every call fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4epi.so")
+
+SWIGLU_INTERLEAVE = 1
+
+# Entry points declared in include/nvfp4epi.h (kept in sync by tests/test_abi.py).
+EXPORTS = (
+    "nvfp4_sf_bytes", "nvfp4_quantize_workspace_bytes", "nvfp4_quantize",
+    "gemm_nvfp4_plain", "gemm_nvfp4_rmsnorm", "gemm_nvfp4_swiglu",
+    "rmsnorm_heads_bf16", "swiglu_bf16", "nvfp4_status_string",
+    "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
+)
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("gscale", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the shared library (once). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libnvfp4epi.so not built at {LIB_PATH}; run __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, vp, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sig = {
+        "nvfp4_sf_bytes": (i64, [i64, i64]),
+        "nvfp4_quantize_workspace_bytes": (i64, []),
+        "nvfp4_quantize": (i32, [vp, i64, i64, i64, i32, i32, _Tensor, vp, vp]),
+        "gemm_nvfp4_plain": (i32, [_Tensor, _Tensor, vp, i64, vp]),
+        "gemm_nvfp4_rmsnorm": (i32, [_Tensor, _Tensor, vp, i32, i64, f32, vp, i64, vp]),
+        "gemm_nvfp4_swiglu": (i32, [_Tensor, _Tensor, vp, i64, ctypes.POINTER(_Tensor), vp]),
+        "rmsnorm_heads_bf16": (i32, [vp, i64, i64, vp, i32, i64, f32, vp, i64, vp]),
+        "swiglu_bf16": (i32, [vp, i64, i64, i64, vp, i64, vp]),
+        "nvfp4_status_string": (ctypes.c_char_p, [i32]),
+        "nvfp4_read_device_status": (i32, [vp]),
+        "nvfp4_selftest_bounded_wait": (i32, [i64, vp]),
+        "nvfp4_launch_count": (i64, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        msg = load().nvfp4_status_string(status).decode()
+        raise RuntimeError(f"{what}: {msg} (status {status})")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+class NVFP4Tensor:
+    """Device buffers of an NVFP4 tensor (see nvfp4_tensor in include/nvfp4epi.h)."""
+
+    def __init__(self, codes: torch.Tensor, sf: torch.Tensor, gscale: torch.Tensor, rows: int, cols: int):
+        self.codes, self.sf, self.gscale, self.rows, self.cols = codes, sf, gscale, rows, cols
+
+    @classmethod
+    def empty(cls, rows: int, cols: int, device="cuda") -> "NVFP4Tensor":
+        return cls(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+                   torch.empty((sf_bytes(rows, cols),), dtype=torch.uint8, device=device),
+                   torch.empty((1,), dtype=torch.float32, device=device), rows, cols)
+
+    def c(self) -> _Tensor:
+        return _Tensor(self.codes.data_ptr(), self.sf.data_ptr(), self.gscale.data_ptr(), self.rows, self.cols)
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.sf.numel() + 4
+
+
+def sf_bytes(rows: int, cols: int) -> int:
+    return int(load().nvfp4_sf_bytes(rows, cols))
+
+
+def quantize_workspace_bytes() -> int:
+    return int(load().nvfp4_quantize_workspace_bytes())
+
+
+def nvfp4_quantize(x: torch.Tensor, out: NVFP4Tensor, compute_amax: bool = True, interleave: bool = False,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> NVFP4Tensor:
+    """Quantise a bf16 2-D CUDA tensor into `out` (see nvfp4_quantize in the header)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    if compute_amax and workspace is None:
+        workspace = torch.empty((quantize_workspace_bytes(),), dtype=torch.uint8, device=x.device)
+    _check(load().nvfp4_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), int(compute_amax),
+                                 SWIGLU_INTERLEAVE if interleave else 0, out.c(), _ptr(workspace),
+                                 _stream(stream)), "nvfp4_quantize")
+    return out
+
+
+def _out2d(D: Optional[torch.Tensor]):
+    if D is None:
+        return None, 0
+    if D.dtype != torch.bfloat16 or D.dim() != 2 or D.stride(1) != 1:
+        raise ValueError("outputs are 2-D bf16 tensors with unit column stride")
+    return D.data_ptr(), D.stride(0)
+
+
+def gemm_nvfp4_plain(A: NVFP4Tensor, B: NVFP4Tensor, D: torch.Tensor, stream=None) -> torch.Tensor:
+    p, ld = _out2d(D)
+    _check(load().gemm_nvfp4_plain(A.c(), B.c(), p, ld, _stream(stream)), "gemm_nvfp4_plain")
+    return D
+
+
+def gemm_nvfp4_rmsnorm(A: NVFP4Tensor, B: NVFP4Tensor, w: Optional[torch.Tensor], head_dim: int,
+                       n_norm_cols: int, eps: float, D: torch.Tensor, stream=None) -> torch.Tensor:
+    if w is not None and (w.dtype != torch.float32 or not w.is_contiguous()):
+        raise ValueError("w must be a contiguous float32 tensor")
+    p, ld = _out2d(D)
+    _check(load().gemm_nvfp4_rmsnorm(A.c(), B.c(), _ptr(w), head_dim, n_norm_cols, eps, p, ld, _stream(stream)),
+           "gemm_nvfp4_rmsnorm")
+    return D
+
+
+def gemm_nvfp4_swiglu(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tensor] = None,
+                      Dq: Optional[NVFP4Tensor] = None, stream=None):
+    p, ld = _out2d(D)
+    dq = ctypes.pointer(Dq.c()) if Dq is not None else None
+    _check(load().gemm_nvfp4_swiglu(A.c(), B.c(), p, ld, dq, _stream(stream)), "gemm_nvfp4_swiglu")
+    return D, Dq
+
+
+def rmsnorm_heads_bf16(x: torch.Tensor, w: torch.Tensor, head_dim: int, n_norm_cols: int, eps: float,
+                       y: torch.Tensor, stream=None) -> torch.Tensor:
+    px, ldx = _out2d(x)
+    py, ldy = _out2d(y)
+    _check(load().rmsnorm_heads_bf16(px, x.shape[0], ldx, w.data_ptr(), head_dim, n_norm_cols, eps, py, ldy,
+                                     _stream(stream)), "rmsnorm_heads_bf16")
+    return y
+
+
+def swiglu_bf16(c: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+    pc, ldc = _out2d(c)
+    py, ldy = _out2d(y)
+    _check(load().swiglu_bf16(pc, c.shape[0], c.shape[1] // 2, ldc, py, ldy, _stream(stream)), "swiglu_bf16")
+    return y
+
+
+def read_device_status(stream=None) -> int:
+    return int(load().nvfp4_read_device_status(_stream(stream)))
+
+
+def selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    _check(load().nvfp4_selftest_bounded_wait(limit_ns, _stream(stream)), "nvfp4_selftest_bounded_wait")
+
+
+def launch_count() -> int:
+    return int(load().nvfp4_launch_count())

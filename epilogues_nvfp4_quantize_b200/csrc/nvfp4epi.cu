@@ -1,0 +1,325 @@
+// C-ABI entry points of libnvfp4epi: argument validation, tensor-map encoding and
+// kernel launches. All device code is in the included headers, built as one
+// translation unit for sm_100a.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "nvfp4epi.h"
+#include "ptx.cuh"
+#include "codec.cuh"
+#include "quantize.cuh"
+#include "unfused.cuh"
+#include "gemm.cuh"
+
+#define NVFP4_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr int kMaxDevices = 64;
+
+std::atomic<int64_t> g_launches{0};
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  bool gemm_attr_set[3] = {false, false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+nvfp4_status current_device(int* dev_out, DeviceInfo** info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NVFP4_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.sm_count = sms;
+    d.probed = true;
+  }
+  if (!d.supported) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+  *dev_out = dev;
+  *info = &d;
+  return NVFP4_OK;
+}
+
+nvfp4_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+nvfp4_status check_operand(const nvfp4_tensor& t) {
+  if (t.codes == nullptr || t.sf == nullptr || t.gscale == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (t.rows <= 0 || t.cols <= 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(t.codes) || !aligned16(t.sf)) return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+// Common checks and launch of the GEMM kernel template.
+template <int EPI>
+nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int64_t ldd, int64_t n_out,
+                      nvfp4::GemmArgs args, cudaStream_t stream) {
+  using namespace nvfp4::gemm_cfg;
+  nvfp4_status st;
+  if ((st = check_operand(A)) != NVFP4_OK) return st;
+  if ((st = check_operand(B)) != NVFP4_OK) return st;
+  const int64_t M = A.rows, K = A.cols, N = B.rows;
+  if (B.cols != K) return NVFP4_ERR_INVALID_ARG;
+  if (M % BM || N % BN || K % BK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (D != nullptr) {
+    if (ldd < n_out) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(D) || (ldd % 8) != 0) return NVFP4_ERR_MISALIGNED;
+  }
+  int dev;
+  DeviceInfo* info;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+
+  CUtensorMap tmA, tmB, tmD;
+  std::memset(&tmD, 0, sizeof(tmD));
+  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.codes, K / 2, M, K / 2, BK_BYTES, BM) ||
+      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B.codes, K / 2, N, K / 2, BK_BYTES, BN))
+    return NVFP4_ERR_CUDA;
+  if (D != nullptr &&
+      !make_map_2d(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, n_out, M, ldd * 2, 64, 32))
+    return NVFP4_ERR_CUDA;
+
+  args.sfa = static_cast<const uint8_t*>(A.sf);
+  args.sfb = static_cast<const uint8_t*>(B.sf);
+  args.ga = A.gscale;
+  args.gb = B.gscale;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.tiles_m = static_cast<int>(M / BM);
+  args.tiles_n = static_cast<int>(N / BN);
+  args.num_tiles = args.tiles_m * args.tiles_n;
+  args.write_d = D != nullptr;
+  args.wait_limit_ns = kWaitLimitNs;
+
+  auto kern = nvfp4::gemm_nvfp4_kernel<EPI>;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->gemm_attr_set[EPI]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      info->gemm_attr_set[EPI] = true;
+    }
+  }
+  const int grid = static_cast<int>(args.num_tiles < info->sm_count ? args.num_tiles : info->sm_count);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmD, args);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+}  // namespace
+
+NVFP4_API int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return -1;
+  return ((rows + 127) / 128) * 128 * ((cols / 16 + 3) / 4) * 4;
+}
+
+NVFP4_API int64_t nvfp4_quantize_workspace_bytes(void) { return 16; }
+
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int compute_amax,
+                                      int flags, nvfp4_tensor out, void* workspace, cudaStream_t stream) {
+  if (x == nullptr || out.codes == nullptr || out.sf == nullptr || out.gscale == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (compute_amax != 0 && compute_amax != 1) return NVFP4_ERR_INVALID_ARG;
+  if (compute_amax && workspace == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~NVFP4_SWIGLU_INTERLEAVE) return NVFP4_ERR_INVALID_ARG;
+  if (out.rows != rows || out.cols != cols) return NVFP4_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || cols % 64 != 0 || ldx < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((flags & NVFP4_SWIGLU_INTERLEAVE) && (rows % 2) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > (1ll << 31) || cols > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx % 8) != 0 || !aligned16(out.codes) ||
+      (reinterpret_cast<uintptr_t>(out.sf) & 3u) != 0 ||
+      (compute_amax && (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  unsigned int* amax = nullptr;
+  if (compute_amax) {
+    amax = static_cast<unsigned int*>(workspace);
+    if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    const int64_t units = rows * (cols / 8);
+    int64_t blocks = (units + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(info->sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    nvfp4::amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(xp, rows, cols, ldx, amax);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if ((st = launch_status()) != NVFP4_OK) return st;
+  }
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t threads = rows_pad * (cols / 8);
+  const int64_t blocks = (threads + 255) / 256;
+  nvfp4::quantize_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      xp, rows, cols, ldx, (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0, amax, out.gscale,
+      static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+NVFP4_API nvfp4_status gemm_nvfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                                        cudaStream_t stream) {
+  if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
+  nvfp4::GemmArgs args{};
+  return run_gemm<nvfp4::EPI_PLAIN>(A, B, D, ldd, B.rows, args, stream);
+}
+
+NVFP4_API nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,
+                                          int64_t n_norm_cols, float eps, void* D, int64_t ldd,
+                                          cudaStream_t stream) {
+  if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (n_norm_cols < 0 || n_norm_cols > B.rows || n_norm_cols % head_dim != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (n_norm_cols > 0 && w == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (w != nullptr && !aligned16(w)) return NVFP4_ERR_MISALIGNED;
+  if (!(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  nvfp4::GemmArgs args{};
+  args.w = w;
+  args.head_dim = head_dim;
+  args.n_norm_cols = static_cast<int>(n_norm_cols);
+  args.eps = eps;
+  return run_gemm<nvfp4::EPI_RMSNORM>(A, B, D, ldd, B.rows, args, stream);
+}
+
+NVFP4_API nvfp4_status gemm_nvfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                                         const nvfp4_tensor* Dq, cudaStream_t stream) {
+  if (D == nullptr && Dq == nullptr) return NVFP4_ERR_INVALID_ARG;
+  const int64_t nh = B.rows / 2;
+  nvfp4::GemmArgs args{};
+  if (Dq != nullptr) {
+    if (Dq->codes == nullptr || Dq->sf == nullptr || Dq->gscale == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (Dq->rows != A.rows || Dq->cols != nh) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(Dq->codes) || !aligned16(Dq->sf)) return NVFP4_ERR_MISALIGNED;
+    args.q_codes = static_cast<uint8_t*>(Dq->codes);
+    args.q_sf = static_cast<uint8_t*>(Dq->sf);
+    args.q_gscale = Dq->gscale;
+    args.q_cols = static_cast<int>(nh);
+  }
+  return run_gemm<nvfp4::EPI_SWIGLU>(A, B, D, ldd, nh, args, stream);
+}
+
+NVFP4_API nvfp4_status rmsnorm_heads_bf16(const void* x, int64_t rows, int64_t ldx, const float* w, int head_dim,
+                                          int64_t n_norm_cols, float eps, void* y, int64_t ldy,
+                                          cudaStream_t stream) {
+  if (x == nullptr || y == nullptr || w == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (head_dim != 128 && head_dim != 256) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows <= 0 || n_norm_cols <= 0 || n_norm_cols % head_dim != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (ldx < n_norm_cols || ldy < n_norm_cols) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(w) || ldx % 8 || ldy % 8) return NVFP4_ERR_MISALIGNED;
+  if (!(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  const int64_t warps = rows * (n_norm_cols / head_dim);
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  if (head_dim == 256)
+    nvfp4::rmsnorm_heads_kernel<256><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(x), rows, ldx, w, n_norm_cols, eps, static_cast<uint16_t*>(y), ldy);
+  else
+    nvfp4::rmsnorm_heads_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(x), rows, ldx, w, n_norm_cols, eps, static_cast<uint16_t*>(y), ldy);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+NVFP4_API nvfp4_status swiglu_bf16(const void* c, int64_t rows, int64_t nh, int64_t ldc, void* y, int64_t ldy,
+                                   cudaStream_t stream) {
+  if (c == nullptr || y == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (rows <= 0 || nh <= 0 || nh % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (ldc < 2 * nh || ldy < nh) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(c) || !aligned16(y) || ldc % 8 || ldy % 8) return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  const int64_t threads = rows * (nh / 8);
+  const int64_t blocks = (threads + 255) / 256;
+  nvfp4::swiglu_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(c), rows, nh, ldc, static_cast<uint16_t*>(y), ldy);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+NVFP4_API const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case NVFP4_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0)";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
+  }
+  return "unknown status";
+}
+
+NVFP4_API int nvfp4_read_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, nvfp4::g_device_status, sizeof(int)) != cudaSuccess) return -1;
+  if (cudaMemcpyToSymbol(nvfp4::g_device_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+NVFP4_API nvfp4_status nvfp4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000ll) return NVFP4_ERR_INVALID_ARG;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  nvfp4::selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_ns));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+NVFP4_API int64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -1,0 +1,181 @@
+/*
+ * nvfp4epi — NVFP4 block-scaled GEMM with its follow-on op fused into the epilogue,
+ * for NVIDIA B200 (sm_100a). C ABI.
+ *
+ * What the library computes follows "Serving sub-second Ideogram v4 without quality
+ * loss" (fal):
+ *   - section "Running the transformer in FP4": FP4 values are E2M1 (1 sign, 2 exponent,
+ *     1 mantissa bit) and the matmul runs natively in 4 bits on Blackwell;
+ *   - section "Epilogue fusion in brief": the GEMM accumulates a tile on chip, and the
+ *     small op that follows (RMSNorm on the attention path, gated SiLU in the FFN) is
+ *     applied before the one store of the output, so no second kernel runs;
+ *   - sections "Tiles and fragments on Blackwell" / "Why head_dim=256 is hard" /
+ *     "Revisit fusion": RMSNorm reduces over a whole head of 128 or 256 columns;
+ *   - section "Fusing gated SiLU (SwiGLU)": output = SiLU(C[:, :N/2]) * C[:, N/2:], with
+ *     the gate/up weight rows interleaved once at packing time;
+ *   - section "Quantization-aware distillation": inference uses static FP4 quantisation,
+ *     so the re-quantised output takes a static per-tensor scale.
+ * The NVFP4 block format (one unsigned E4M3 scale per 16 elements along K, one FP32
+ * scale per tensor) is the format those kernels consume; the page names NVFP4 without
+ * spelling out the block size.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller. The library never
+ *     allocates device memory.
+ *   - Every call is asynchronous on the given stream; nothing synchronises.
+ *   - Argument and shape errors return a status synchronously and launch nothing.
+ *     CUDA launch errors return NVFP4_ERR_CUDA. There is no exception, no abort and no
+ *     device assert. Every wait inside a kernel is bounded in time; a wait that runs
+ *     out records NVFP4_ERR_DEVICE_TIMEOUT in a device status word, read with
+ *     nvfp4_read_device_status().
+ *   - Only compute capability 10.0 (B200) is supported (NVFP4_ERR_UNSUPPORTED_DEVICE).
+ *   - bf16 tensors are row-major with a leading dimension given in elements.
+ */
+#ifndef NVFP4EPI_H
+#define NVFP4EPI_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, bad flag, inconsistent sizes */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size rule below is not met */
+  NVFP4_ERR_MISALIGNED = 3,        /* a pointer or leading dimension is not 16-byte aligned */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 4,
+  NVFP4_ERR_CUDA = 5,
+  NVFP4_ERR_DEVICE_TIMEOUT = 6
+} nvfp4_status;
+
+/*
+ * An NVFP4 tensor of rows x cols logical elements, quantised in blocks of 16 adjacent
+ * elements along cols (the K axis of a GEMM operand, the N axis of an output).
+ *   codes : rows x cols/2 bytes, row-major, row stride cols/2 bytes. Byte j of a row holds
+ *           element 2j in bits 0-3 and element 2j+1 in bits 4-7 (E2M1 codes: s e1 e0 m).
+ *   sf    : nvfp4_sf_bytes(rows, cols) bytes of unsigned E4M3 block scales in the
+ *           tensor-core scale layout: the scales of each 128-row x 4-block tile form one
+ *           512-byte unit, units ordered by row tile then by 4-block group, and inside a
+ *           unit row r, block c sits at byte (r % 32) * 16 + (r / 32) * 4 + c.
+ *   gscale: device pointer to the FP32 per-tensor scale G. Element i of block b decodes
+ *           to e2m1(code_i) * e4m3(sf_b) * G.
+ */
+typedef struct {
+  void* codes;
+  void* sf;
+  float* gscale;
+  int64_t rows;
+  int64_t cols;
+} nvfp4_tensor;
+
+/* Bytes of the block-scale buffer: rows padded to 128, 16-blocks padded to 4. */
+int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of device scratch nvfp4_quantize needs when it derives G itself. */
+int64_t nvfp4_quantize_workspace_bytes(void);
+
+/* Pack-time row permutation for the SwiGLU weight (section "Fusing gated SiLU"). */
+#define NVFP4_SWIGLU_INTERLEAVE 1
+
+/*
+ * Quantise a bf16 tensor x (rows x cols, leading dimension ldx elements) to NVFP4.
+ *   compute_amax = 1: G = amax(|x|) / (6 * 448) is computed on the device and written to
+ *                     *out.gscale; `workspace` must hold
+ *                     nvfp4_quantize_workspace_bytes() bytes (contents on entry ignored).
+ *   compute_amax = 0: *out.gscale is used as given (static scale, must be > 0 and finite);
+ *                     workspace may be NULL.
+ * Per block of 16, in IEEE float32: s = E4M3_rn_satfinite(amax_b * (1 / (6 G))) (s = 0
+ * for an all-zero block), d = e4m3(s) * G, q_i = E2M1_rn_satfinite(x_i * (1 / d)) (q = 0
+ * when d = 0).
+ * flags: 0, or NVFP4_SWIGLU_INTERLEAVE: x is a [gate | up] weight of 2*Nh rows and output
+ *        row 2j takes input row j, row 2j+1 takes input row Nh + j.
+ * Rules: rows >= 1 (even with the interleave flag), cols % 64 == 0, ldx >= cols,
+ *        x and ldx*2 bytes 16-byte aligned, out.rows == rows, out.cols == cols,
+ *        out.codes 16-byte aligned, out.sf 4-byte aligned. Padding scale bytes are
+ *        written as 0.
+ */
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                            int compute_amax, int flags, nvfp4_tensor out,
+                            void* workspace, cudaStream_t stream);
+
+/*
+ * D (M x N bf16, leading dimension ldd) = bf16(G_A * G_B * sum_k A[m,k] * B[n,k]) with
+ * A (M x K) and B (N x K) NVFP4, both K-contiguous.
+ * Rules: M % 128 == 0, N % 256 == 0, K % 256 == 0, A.cols == B.cols == K,
+ *        ldd >= N, ldd % 8 == 0, every pointer 16-byte aligned.
+ */
+nvfp4_status gemm_nvfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                              cudaStream_t stream);
+
+/*
+ * As gemm_nvfp4_plain, then per row and per head of head_dim adjacent columns among the
+ * first n_norm_cols: y = x * rsqrt(mean(x^2) + eps) * w[col] (x = G_A G_B acc, float32);
+ * columns >= n_norm_cols pass through (the V block of a QKV projection).
+ *   w: n_norm_cols float32 weights, one per normalised column (a head_dim-long weight
+ *      shared by the heads of a block is expanded by the caller).
+ * Rules: the plain rules, head_dim in {128, 256}, n_norm_cols % head_dim == 0,
+ *        n_norm_cols <= N, w 16-byte aligned (may be NULL only if n_norm_cols == 0).
+ */
+nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w,
+                                int head_dim, int64_t n_norm_cols, float eps,
+                                void* D, int64_t ldd, cudaStream_t stream);
+
+/*
+ * SwiGLU epilogue. B is the gate|up weight (N = 2*Nh rows) packed with
+ * NVFP4_SWIGLU_INTERLEAVE, so accumulator columns come as [g0, u0, g1, u1, ...].
+ *   out[m, j] = silu(x_g) * x_u, silu(x) = x / (1 + exp(-x)), x = G_A G_B acc.
+ *   D  : M x Nh bf16 output (leading dimension ldd), or NULL.
+ *   Dq : M x Nh NVFP4 output quantised from the bf16-rounded values with the static
+ *        scale *Dq->gscale (the rule of nvfp4_quantize with compute_amax = 0), or NULL.
+ *        Its layout is the A-operand layout of the next GEMM (K = Nh).
+ * At least one of D and Dq is given. Rules: the plain rules with Nh = N/2 in place of N
+ * for ldd; Dq->rows == M, Dq->cols == Nh.
+ */
+nvfp4_status gemm_nvfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                               const nvfp4_tensor* Dq, cudaStream_t stream);
+
+/*
+ * Unfused comparison ops (a GEMM writes its bf16 output; a second kernel applies the op).
+ * rmsnorm_heads_bf16: y[:, :n_norm_cols] = per-head RMSNorm of x[:, :n_norm_cols] with
+ *   the same formula as gemm_nvfp4_rmsnorm; other columns of y are not touched. y may
+ *   equal x (in place). Rules: head_dim in {128, 256}, n_norm_cols % head_dim == 0,
+ *   ldx, ldy >= n_norm_cols, 16-byte aligned rows.
+ * swiglu_bf16: y (rows x nh) = silu(c[:, :nh]) * c[:, nh:2nh] for c of rows x 2nh
+ *   (logical [gate | up] columns). Rules: nh % 8 == 0, ldc >= 2nh, ldy >= nh, 16-byte
+ *   aligned rows.
+ */
+nvfp4_status rmsnorm_heads_bf16(const void* x, int64_t rows, int64_t ldx, const float* w,
+                                int head_dim, int64_t n_norm_cols, float eps,
+                                void* y, int64_t ldy, cudaStream_t stream);
+nvfp4_status swiglu_bf16(const void* c, int64_t rows, int64_t nh, int64_t ldc,
+                         void* y, int64_t ldy, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* nvfp4_status_string(nvfp4_status status);
+
+/*
+ * Synchronise `stream`, return the device status word of the current device (0 or an
+ * nvfp4_status recorded by a kernel whose bounded wait ran out) and clear it.
+ * Returns -1 if the read itself failed.
+ */
+int nvfp4_read_device_status(cudaStream_t stream);
+
+/*
+ * Self-test of the bounded-wait path: launches one block that waits on a barrier that
+ * nothing completes, giving up after limit_ns nanoseconds (1 <= limit_ns <= 1e9).
+ * The kernel then records NVFP4_ERR_DEVICE_TIMEOUT in the device status word and
+ * returns normally, leaving the context usable.
+ */
+nvfp4_status nvfp4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream);
+
+/* Number of kernels the library has launched in this process (for launch accounting). */
+int64_t nvfp4_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4EPI_H */

@@ -58,6 +58,7 @@ def e2m1_decode(codes) -> np.ndarray:
 
 
 _E2M1_MAGS = e2m1_decode(np.arange(8))          # increasing in the code
+_E2M1_TABLE = e2m1_decode(np.arange(16))         # code -> value lookup
 
 
 def _rne_to_table(ax: np.ndarray, table: np.ndarray) -> np.ndarray:
@@ -80,11 +81,21 @@ def _rne_to_table(ax: np.ndarray, table: np.ndarray) -> np.ndarray:
 
 def e2m1_encode(x) -> np.ndarray:
     """float32 -> E2M1 code, round to nearest with ties to the even mantissa,
-    saturating at +-6. The sign bit follows the input's sign bit (so -0.1 -> 0x8)."""
+    saturating at +-6. The sign bit follows the input's sign bit (so -0.1 -> 0x8).
+
+    The magnitude index is the number of midpoints between adjacent levels that |x|
+    lies above; at a midpoint exactly, the even index of the two neighbours wins.
+    (Every midpoint is exact in float32, so the comparisons are exact.)
+    """
     x = np.asarray(x, dtype=F32)
-    ax = np.abs(x).astype(np.float64)
-    idx = _rne_to_table(ax, _E2M1_MAGS)
-    return (idx | (np.signbit(x).astype(np.int64) << 3)).astype(np.uint8)
+    ax = np.abs(x)
+    idx = np.zeros(x.shape, np.uint8)
+    for i in range(7):
+        mid = F32((_E2M1_MAGS[i] + _E2M1_MAGS[i + 1]) / 2)
+        idx += (ax > mid)
+        if (i + 1) % 2 == 0:
+            idx += (ax == mid)
+    return idx | (np.signbit(x).astype(np.uint8) << 3)
 
 
 # ----------------------------------------------------------------------------------
@@ -106,6 +117,7 @@ def e4m3_decode(codes) -> np.ndarray:
 
 
 _E4M3_MAGS = e4m3_decode(np.arange(0x7F))       # codes 0x00..0x7E, increasing
+_E4M3_TABLE = e4m3_decode(np.arange(256))        # code -> value lookup
 
 
 def e4m3_encode(x) -> np.ndarray:
@@ -169,8 +181,9 @@ def dequantize(codes, scales, G) -> np.ndarray:
     """dec(q) * dec(s) * G in float64, (rows, cols)."""
     codes = np.asarray(codes)
     rows, cols = codes.shape
-    sc = np.repeat(e4m3_decode(scales), BLOCK, axis=1)
-    return e2m1_decode(codes) * sc * float(G)
+    vals = _E2M1_TABLE[codes & 0xF].reshape(rows, cols // BLOCK, BLOCK)
+    vals *= (_E4M3_TABLE[np.asarray(scales)] * float(G))[:, :, None]
+    return vals.reshape(rows, cols)
 
 
 # ----------------------------------------------------------------------------------
@@ -324,29 +337,35 @@ def quantized_operand(x_bf16):
     return quantize(_as_f32(x_bf16))
 
 
-def problem_gemm(a_bf16, b_bf16, rows=None) -> np.ndarray:
-    """float64 C = dequant(A) @ dequant(B)^T, optionally only for the given rows of A
-    (G of A is still the whole tensor's)."""
-    qa, sa, ga = quantized_operand(a_bf16)
-    qb, sb, gb = quantized_operand(b_bf16)
-    a = dequantize(qa, sa, ga)
+def problem_gemm(a_bf16, b_bf16, rows=None, b_quant=None) -> np.ndarray:
+    """float64 C = dequant(A) @ dequant(B)^T.
+
+    rows: optionally only these rows of A. Quantisation is row-local once G is fixed,
+    so the rows are quantised with the whole tensor's G (identical to quantising all of
+    A and keeping those rows).
+    b_quant: optionally the (codes, scales, G) of B from an earlier quantized_operand(b).
+    """
+    a = _as_f32(a_bf16)
+    Ga = global_scale(a)
     if rows is not None:
-        a = a[rows]
-    return gemm(a, dequantize(qb, sb, gb))
+        a = a[np.asarray(rows)]
+    qa, sa, _ = quantize(a, Ga)
+    qb, sb, gb = quantized_operand(b_bf16) if b_quant is None else b_quant
+    return gemm(dequantize(qa, sa, Ga), dequantize(qb, sb, gb))
 
 
-def problem_plain(a_bf16, b_bf16, rows=None) -> np.ndarray:
-    return bf16_round(problem_gemm(a_bf16, b_bf16, rows))
+def problem_plain(a_bf16, b_bf16, rows=None, b_quant=None) -> np.ndarray:
+    return bf16_round(problem_gemm(a_bf16, b_bf16, rows, b_quant))
 
 
-def problem_rmsnorm(a_bf16, b_bf16, w, head_dim, n_norm_cols, eps, rows=None) -> np.ndarray:
-    c = problem_gemm(a_bf16, b_bf16, rows)
+def problem_rmsnorm(a_bf16, b_bf16, w, head_dim, n_norm_cols, eps, rows=None, b_quant=None) -> np.ndarray:
+    c = problem_gemm(a_bf16, b_bf16, rows, b_quant)
     return bf16_round(rmsnorm_heads(c, w, head_dim, n_norm_cols, eps))
 
 
-def problem_swiglu(a_bf16, b_gate_up_bf16, rows=None) -> np.ndarray:
+def problem_swiglu(a_bf16, b_gate_up_bf16, rows=None, b_quant=None) -> np.ndarray:
     """b_gate_up is the logical [gate | up] weight (2*Nh x K)."""
-    return bf16_round(swiglu(problem_gemm(a_bf16, b_gate_up_bf16, rows)))
+    return bf16_round(swiglu(problem_gemm(a_bf16, b_gate_up_bf16, rows, b_quant)))
 
 
 def requantize(out_bf16_values, G):

@@ -1,0 +1,194 @@
+"""GPU parity of the fused GEMM entry points against the oracle, at sizes the oracle
+finishes in seconds that still span several tiles, several tiles per CTA, and the
+degenerate cases (one tile, one K step, no normalised columns)."""
+import numpy as np
+import pytest
+import torch
+
+import epilogues_nvfp4_quantize_b200 as ep
+from oracle import nvfp4_oracle as o
+import workloads as wk
+from gpu_util import (assert_close, bf16_bits, bf16_to_np, device, nvfp4_from_arrays, quantize_gpu,
+                      read_nvfp4, rel_err, REL_TOL)
+
+pytestmark = pytest.mark.gpu
+
+
+def _exact_operands(M, N, K, seed):
+    qa = wk.fp4_codes_exact(M, K, seed, 21)
+    qb = wk.fp4_codes_exact(N, K, seed, 22)
+    sa = o.e4m3_encode(wk.pow2_scales_exact(M, K // 16, seed, 23).astype(np.float32))
+    sb = o.e4m3_encode(wk.pow2_scales_exact(N, K // 16, seed, 24).astype(np.float32))
+    return qa, sa, qb, sb
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 1024), (384, 768, 3072), (2048, 2560, 256)])
+def test_plain_gemm_is_exact_on_exactly_representable_inputs(M, N, K):
+    """E2M1 codes x power-of-two scales: every partial sum is a multiple of 2^-6 below
+    2^24 * 2^-6, so FP32 accumulation is exact in any order and the bf16 output must be
+    the round-to-nearest-even of the exact product, bit for bit. This pins the operand
+    layout, the scale-factor layout and the MMA kind."""
+    qa, sa, qb, sb = _exact_operands(M, N, K, seed=M + N + K)
+    A = nvfp4_from_arrays(qa, sa, 1.0)
+    B = nvfp4_from_arrays(qb, sb, 1.0)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_plain(A, B, D)
+    ref = o.bf16_round(o.gemm(o.dequantize(qa, sa, 1.0), o.dequantize(qb, sb, 1.0)))
+    got = bf16_bits(D)
+    want = o.bf16_bits(ref)
+    assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} outputs differ"
+
+
+def test_plain_gemm_scales_by_both_global_scales():
+    M, N, K = 128, 256, 512
+    qa, sa, qb, sb = _exact_operands(M, N, K, seed=5)
+    A = nvfp4_from_arrays(qa, sa, 0.5)
+    B = nvfp4_from_arrays(qb, sb, 0.25)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_plain(A, B, D)
+    ref = o.bf16_round(o.gemm(o.dequantize(qa, sa, 0.5), o.dequantize(qb, sb, 0.25)))
+    assert np.array_equal(bf16_bits(D), o.bf16_bits(ref))
+
+
+@pytest.mark.parametrize("M,N,K,ldd", [(256, 512, 512, 512), (1280, 768, 768, 800), (2048, 2560, 512, 2560)])
+def test_plain_gemm_matches_oracle(M, N, K, ldd):
+    a = wk.activations(M, K, wk.outlier_count(K), seed=1)
+    b = wk.weights(N, K, 1 / np.sqrt(K), seed=1)
+    A, B = quantize_gpu(a), quantize_gpu(b)
+    Dfull = torch.full((M, ldd), 7.0, dtype=torch.bfloat16, device=device())
+    D = Dfull[:, :N]
+    ep.gemm_nvfp4_plain(A, B, D)
+    assert_close(bf16_to_np(D), o.problem_plain(a, b), "plain")
+    if ldd > N:  # the columns past N of each row are untouched
+        assert torch.all(Dfull[:, N:] == 7.0)
+
+
+def _rmsnorm_case(M, K, N, hd, n_norm, seed=0, eps=1e-6):
+    a = wk.activations(M, K, wk.outlier_count(K), seed=seed)
+    b = wk.weights(N, K, 1 / np.sqrt(K), seed=seed)
+    w = np.tile(wk.norm_weight(hd, seed), max(n_norm // hd, 1))[:n_norm].astype(np.float32)
+    A, B = quantize_gpu(a), quantize_gpu(b)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    wt = torch.from_numpy(w).to(device()) if n_norm else None
+    ep.gemm_nvfp4_rmsnorm(A, B, wt, hd, n_norm, eps, D)
+    ref = o.problem_rmsnorm(a, b, w, hd, n_norm, eps)
+    return bf16_to_np(D), ref
+
+
+@pytest.mark.parametrize("M,K,N,hd,n_norm", [
+    (256, 1024, 1024, 256, 1024),   # the tiny QK-norm case: 4 heads of 256, all normalised
+    (256, 512, 768, 256, 512),      # V block passes through
+    (256, 512, 768, 128, 384),      # 128-wide heads, normalised part ends mid-tile
+    (384, 256, 512, 128, 0),        # nothing normalised
+    (2048, 512, 2560, 256, 1536),   # several tiles per CTA
+])
+def test_rmsnorm_gemm_matches_oracle(M, K, N, hd, n_norm):
+    got, ref = _rmsnorm_case(M, K, N, hd, n_norm)
+    assert_close(got, ref, f"rmsnorm hd{hd}")
+
+
+def test_rmsnorm_output_has_unit_rms_per_head_before_weight():
+    M, K, N, hd = 256, 512, 512, 256
+    a = wk.activations(M, K, 1, seed=3)
+    b = wk.weights(N, K, 1 / np.sqrt(K), seed=3)
+    A, B = quantize_gpu(a), quantize_gpu(b)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_rmsnorm(A, B, torch.ones(N, device=device()), hd, N, 0.0, D)
+    y = bf16_to_np(D).reshape(M, N // hd, hd)
+    rms = np.sqrt(np.mean(y * y, axis=2))
+    np.testing.assert_allclose(rms, 1.0, rtol=4e-3)
+
+
+def _swiglu_case(M, K, nh, seed=0, requant=True, write_d=True):
+    a = wk.activations(M, K, wk.outlier_count(K), seed=seed)
+    b = wk.weights(2 * nh, K, 1 / np.sqrt(K), seed=seed)     # logical [gate | up]
+    A = quantize_gpu(a)
+    B = quantize_gpu(b, interleave=True)
+    ref = o.problem_swiglu(a, b)
+    G = np.float32(np.abs(ref).max() / 2688)                 # static scale of the output
+    D = torch.empty(M, nh, dtype=torch.bfloat16, device=device()) if write_d else None
+    Dq = None
+    if requant:
+        Dq = ep.NVFP4Tensor.empty(M, nh, device())
+        Dq.gscale.fill_(float(G))
+    ep.gemm_nvfp4_swiglu(A, B, D, Dq)
+    return a, b, ref, G, D, Dq
+
+
+@pytest.mark.parametrize("M,K,nh", [(128, 256, 128), (256, 512, 512), (2048, 512, 1280)])
+def test_swiglu_gemm_matches_oracle(M, K, nh):
+    a, b, ref, G, D, Dq = _swiglu_case(M, K, nh)
+    got = bf16_to_np(D)
+    assert_close(got, ref, "swiglu")
+    # re-quantised output, code for code against the oracle's re-quantisation of its
+    # own bf16 result: a differing code is allowed only where the two bf16 values differ,
+    # and then by at most one level
+    q_ref, s_ref, _ = o.requantize(ref, G)
+    q, s, Gq, _ = read_nvfp4(Dq)
+    assert Gq == G
+    same_bf16 = np.repeat((got == ref).reshape(M, nh // 16, 16).all(axis=2), 16, axis=1)
+    code_diff = q != q_ref
+    assert not (code_diff & same_bf16).any()
+    blk_same = (got == ref).reshape(M, nh // 16, 16).all(axis=2)
+    assert np.array_equal(s[blk_same], s_ref[blk_same])
+    lv = np.abs(o.e2m1_decode(q) - o.e2m1_decode(q_ref))
+    assert code_diff.mean() < 0.01
+    assert np.all(lv[code_diff] <= 2.0)
+
+
+def test_fused_requant_equals_quantize_of_fused_bf16():
+    """GPU invariant: the re-quantised output is nvfp4_quantize (static scale) applied to
+    the fused bf16 output, bit for bit."""
+    a, b, ref, G, D, Dq = _swiglu_case(512, 768, 768, seed=4)
+    t = ep.NVFP4Tensor.empty(512, 768, device())
+    t.gscale.fill_(float(G))
+    ep.nvfp4_quantize(D, t, compute_amax=False)
+    q1, s1, _, b1 = read_nvfp4(Dq)
+    q2, s2, _, b2 = read_nvfp4(t)
+    assert np.array_equal(q1, q2) and np.array_equal(b1, b2)
+
+
+def test_swiglu_requant_only():
+    a, b, ref, G, D, Dq = _swiglu_case(256, 256, 256, seed=6, write_d=False)
+    q_ref, s_ref, _ = o.requantize(ref, G)
+    q, s, _, _ = read_nvfp4(Dq)
+    deq = o.dequantize(q, s, G)
+    deq_ref = o.dequantize(q_ref, s_ref, G)
+    assert np.linalg.norm(deq - deq_ref) / np.linalg.norm(deq_ref) < 1e-2
+
+
+def test_unfused_ops_match_oracle():
+    M, N, hd, nn = 256, 1024, 256, 768
+    x = wk.activations(M, N, 0, seed=8)
+    w = np.tile(wk.norm_weight(hd, 8), nn // hd).astype(np.float32)
+    xd = x.to(device())
+    y = xd.clone()
+    ep.rmsnorm_heads_bf16(xd, torch.from_numpy(w).to(device()), hd, nn, 1e-6, y)
+    ref = o.bf16_round(o.rmsnorm_heads(x.double().numpy(), w, hd, nn, 1e-6))
+    assert_close(bf16_to_np(y), ref, "rmsnorm_heads_bf16")
+    for hd2 in (128,):
+        y2 = torch.empty_like(xd)
+        w2 = np.tile(wk.norm_weight(hd2, 9), N // hd2).astype(np.float32)
+        ep.rmsnorm_heads_bf16(xd, torch.from_numpy(w2).to(device()), hd2, N, 1e-6, y2)
+        ref2 = o.bf16_round(o.rmsnorm_heads(x.double().numpy(), w2, hd2, N, 1e-6))
+        assert_close(bf16_to_np(y2), ref2, "rmsnorm_heads_bf16 hd128")
+    c = wk.activations(M, 2 * 512, 0, seed=10).to(device())
+    ys = torch.empty(M, 512, dtype=torch.bfloat16, device=device())
+    ep.swiglu_bf16(c, ys)
+    refs = o.bf16_round(o.swiglu(c.double().cpu().numpy()))
+    assert_close(bf16_to_np(ys), refs, "swiglu_bf16")
+
+
+def test_bounded_wait_times_out_into_a_status_and_the_context_survives():
+    assert ep.read_device_status() == 0
+    ep.selftest_bounded_wait(2_000_000)  # 2 ms
+    assert ep.read_device_status() == 6
+    assert ep.read_device_status() == 0  # reading clears it
+    # the context is still usable
+    got, ref = _rmsnorm_case(128, 256, 256, 128, 256, seed=2)
+    assert_close(got, ref, "after timeout")
+
+
+def test_no_device_errors_recorded():
+    torch.cuda.synchronize()
+    assert ep.read_device_status() == 0
