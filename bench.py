@@ -1,0 +1,487 @@
+"""Benchmark of the NVFP4 GEMM + fused-epilogue hot path on B200.
+
+One step = one DiT layer's projection path over M tokens, all on the GPU through the
+C ABI (weights packed once beforehand, untimed):
+  1. nvfp4_quantize(x)                    activations 16384 x 3072 bf16 -> NVFP4 (amax pass + quantise)
+  2. gemm_nvfp4_rmsnorm(x, Wqkv)          N = 9216 (12 heads x 256 for each of Q, K, V),
+                                          RMSNorm head_dim 256 on Q and K, V passed through
+  3. gemm_nvfp4_swiglu(x, Wup) -> h       N = 2 x 12288 gate|up, SwiGLU, NVFP4 re-quantisation
+                                          with a static scale (calibrated once, untimed)
+  4. gemm_nvfp4_plain(h, Wdown)           K = 12288, N = 3072
+value = GEMM FLOPs of the step (2MNK summed over the three GEMMs) / step time, TFLOP/s.
+Separately timed (not in `value`): the unfused comparison (plain GEMM writes bf16, then a
+separate RMSNorm / SwiGLU / quantise kernel), reported as fused-vs-unfused speedups.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own M-token batch, no
+collective on the data path (weak scaling); time = max over ranks.
+
+--impl reference times the CPU oracle (oracle/) on a bounded row sample of the same step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "fused NVFP4 GEMM+epilogue TFLOPS and % of B200 FP4 peak; fused-vs-unfused speedup"
+K_IN, N_QKV, N_NORM, HD, N_UP, K_DOWN = 3072, 9216, 6144, 256, 24576, 12288
+EPS = 1e-6
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+
+
+def step_flops(M: int) -> dict:
+    return {"qkv": 2 * M * N_QKV * K_IN, "up": 2 * M * N_UP * K_IN, "down": 2 * M * K_DOWN * K_IN}
+
+
+def workload_desc(M: int) -> str:
+    return (f"DiT layer projections at M={M} tokens: quantise x ({M}x{K_IN} bf16) -> QKV GEMM "
+            f"N={N_QKV} + per-head RMSNorm hd{HD} on Q,K (V passthrough) -> FFN-up GEMM N={N_UP} "
+            f"SwiGLU + NVFP4 re-quantisation -> FFN-down GEMM K={K_DOWN} N={K_IN}")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join("/tmp", f"nvfp4_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, pw, reasons = [], 0.0, [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                s = float(parts[1].split()[0])
+                mx = max(mx, float(parts[2].split()[0]))
+                w = float(parts[3].split()[0])
+            except ValueError:
+                continue
+            sm.append(s)
+            pw.append(w)
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        loaded = [s for s, w in zip(sm, pw) if w > 0.5 * max(pw)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(pw)}
+
+
+# ----------------------------------------------------------------------------------
+# the CUDA arm
+# ----------------------------------------------------------------------------------
+class Layer:
+    """Device-resident weights and activations of one DiT layer's projections."""
+
+    def __init__(self, M: int, dev, seed: int):
+        import torch
+        import epilogues_nvfp4_quantize_b200 as ep
+        import workloads as wk
+        self.M, self.dev = M, dev
+        T = ep.NVFP4Tensor
+        self.x = wk.activations(M, K_IN, wk.outlier_count(K_IN), seed=seed).to(dev)
+        std = 1.0 / np.sqrt(K_IN)
+        w_qkv = wk.weights(N_QKV, K_IN, std, seed=seed, stream=11).to(dev)
+        w_up = wk.weights(N_UP, K_IN, std, seed=seed, stream=12).to(dev)
+        w_down = wk.weights(K_IN, K_DOWN, 1.0 / np.sqrt(K_DOWN), seed=seed, stream=13).to(dev)
+        # weight packing (offline): quantise, SwiGLU interleave of the gate|up rows
+        self.Wqkv, self.Wup, self.Wup_logical, self.Wdown = (T.empty(N_QKV, K_IN, dev), T.empty(N_UP, K_IN, dev),
+                                                             T.empty(N_UP, K_IN, dev), T.empty(K_IN, K_DOWN, dev))
+        ep.nvfp4_quantize(w_qkv, self.Wqkv)
+        ep.nvfp4_quantize(w_up, self.Wup, interleave=True)
+        ep.nvfp4_quantize(w_up, self.Wup_logical)
+        ep.nvfp4_quantize(w_down, self.Wdown)
+        wq = wk.norm_weight(HD, seed, 3)
+        wkk = wk.norm_weight(HD, seed, 5)
+        self.w_norm = torch.from_numpy(np.concatenate([np.tile(wq, N_NORM // 2 // HD),
+                                                       np.tile(wkk, N_NORM // 2 // HD)]).astype(np.float32)).to(dev)
+        del w_qkv, w_up, w_down
+        self.ws = torch.empty(ep.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+        self.xq = T.empty(M, K_IN, dev)
+        self.qkv = torch.empty(M, N_QKV, dtype=torch.bfloat16, device=dev)
+        self.h = T.empty(M, N_UP // 2, dev)
+        self.out = torch.empty(M, K_IN, dtype=torch.bfloat16, device=dev)
+        # static scale of the re-quantised FFN activations: calibrated once from a bf16
+        # run of the fused SwiGLU GEMM (amax / 2688, derived by the library's quantiser)
+        ep.nvfp4_quantize(self.x, self.xq, workspace=self.ws)
+        hb = torch.empty(M, N_UP // 2, dtype=torch.bfloat16, device=dev)
+        ep.gemm_nvfp4_swiglu(self.xq, self.Wup, hb, None)
+        ep.nvfp4_quantize(hb, self.h, workspace=self.ws)
+        torch.cuda.synchronize(dev)
+        del hb
+
+    def step(self, ev=None):
+        import epilogues_nvfp4_quantize_b200 as ep
+        ep.nvfp4_quantize(self.x, self.xq, workspace=self.ws)
+        if ev is not None:
+            ev[0].record()
+        ep.gemm_nvfp4_rmsnorm(self.xq, self.Wqkv, self.w_norm, HD, N_NORM, EPS, self.qkv)
+        if ev is not None:
+            ev[1].record()
+        ep.gemm_nvfp4_swiglu(self.xq, self.Wup, None, self.h)
+        if ev is not None:
+            ev[2].record()
+        ep.gemm_nvfp4_plain(self.h, self.Wdown, self.out)
+
+    # unfused comparison: GEMM -> bf16 in HBM -> separate op kernel(s)
+    def alloc_unfused(self):
+        import torch
+        import epilogues_nvfp4_quantize_b200 as ep
+        self.c_up = torch.empty(self.M, N_UP, dtype=torch.bfloat16, device=self.dev)
+        self.y_up = torch.empty(self.M, N_UP // 2, dtype=torch.bfloat16, device=self.dev)
+        self.h2 = ep.NVFP4Tensor(torch.empty_like(self.h.codes), torch.empty_like(self.h.sf), self.h.gscale,
+                                 self.h.rows, self.h.cols)
+
+    def unfused_qkv(self):
+        import epilogues_nvfp4_quantize_b200 as ep
+        ep.gemm_nvfp4_plain(self.xq, self.Wqkv, self.qkv)
+        ep.rmsnorm_heads_bf16(self.qkv, self.w_norm, HD, N_NORM, EPS, self.qkv)
+
+    def unfused_up(self):
+        import epilogues_nvfp4_quantize_b200 as ep
+        ep.gemm_nvfp4_plain(self.xq, self.Wup_logical, self.c_up)
+        ep.swiglu_bf16(self.c_up, self.y_up)
+        ep.nvfp4_quantize(self.y_up, self.h2, compute_amax=False)
+
+
+def time_loop(fn, steps, warmup, torch):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+    import epilogues_nvfp4_quantize_b200 as ep
+    from epilogues_nvfp4_quantize_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    ep.load()
+
+    M = args.M
+    layer = Layer(M, dev, seed=rank)
+    flops = step_flops(M)
+    total_flops = sum(flops.values())
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        layer.step()
+    barrier()
+
+    # ---- timed region: K back-to-back steps (inputs x + weights exceed the L2)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    n0 = ep.launch_count()
+    with ClockSampler(local) as clk:
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for i in range(K):
+            ev_s[i].record()
+            layer.step(ev[i])
+            ev_e[i].record()
+        stop.record()
+        torch.cuda.synchronize(dev)
+    launches = ep.launch_count() - n0
+    ms_total = start.elapsed_time(stop)
+    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / K
+    per = {"quantize_x": [], "qkv_rmsnorm": [], "up_swiglu_requant": [], "down_plain": []}
+    for i in range(K):
+        per["quantize_x"].append(ev_s[i].elapsed_time(ev[i][0]))
+        per["qkv_rmsnorm"].append(ev[i][0].elapsed_time(ev[i][1]))
+        per["up_swiglu_requant"].append(ev[i][1].elapsed_time(ev[i][2]))
+        per["down_plain"].append(ev[i][2].elapsed_time(ev_e[i]))
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    value = total_flops * world / (ms_total / K * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    pk = peaks()
+    fp4_peak = pk["bf16"] * FP4_PER_BF16
+    up_tflops = flops["up"] / (avg["up_swiglu_requant"] * 1e-3) / 1e12
+    kernels = {
+        "quantize_x": {"us": avg["quantize_x"] * 1e3,
+                       "gbs": (M * K_IN * 2 + M * K_IN * (0.5 + 1 / 16)) / (avg["quantize_x"] * 1e-3) / 1e9},
+        "qkv_rmsnorm": {"us": avg["qkv_rmsnorm"] * 1e3,
+                        "tflops": flops["qkv"] / (avg["qkv_rmsnorm"] * 1e-3) / 1e12},
+        "up_swiglu_requant": {"us": avg["up_swiglu_requant"] * 1e3, "tflops": up_tflops},
+        "down_plain": {"us": avg["down_plain"] * 1e3,
+                       "tflops": flops["down"] / (avg["down_plain"] * 1e-3) / 1e12},
+    }
+    for k in ("qkv_rmsnorm", "up_swiglu_requant", "down_plain"):
+        kernels[k]["pct_fp4_peak"] = 100.0 * kernels[k]["tflops"] / fp4_peak
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": workload_desc(M), "M": M, "K": K_IN, "N_qkv": N_QKV, "N_up": N_UP,
+                   "K_down": K_DOWN, "head_dim": HD, "global_batch_tokens": M * world,
+                   "parallelism": f"dp{world} (independent token batches, no collective)",
+                   "l2": "no flush: per-step inputs (x 100.7 MB + packed weights 75 MB) exceed the 126 MB L2"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel<SWIGLU> (FFN-up, requant)",
+                     "achieved": round(up_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(up_tflops / fp4_peak, 4), "traffic": args.traffic,
+                     "peak_source": f"{pk['source']} bf16 {pk['bf16']} TFLOP/s x {FP4_PER_BF16} (nominal dense "
+                                    f"FP4:BF16 ratio), burst figure"},
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+
+    # ---- unfused comparison (separately timed, same step shapes)
+    if not args.no_unfused:
+        layer.alloc_unfused()
+        barrier()
+        t_fused_qkv = time_loop(lambda: ep.gemm_nvfp4_rmsnorm(layer.xq, layer.Wqkv, layer.w_norm, HD, N_NORM, EPS,
+                                                              layer.qkv), args.cmp_steps, 3, torch)
+        t_unf_qkv = time_loop(layer.unfused_qkv, args.cmp_steps, 3, torch)
+        t_fused_up = time_loop(lambda: ep.gemm_nvfp4_swiglu(layer.xq, layer.Wup, None, layer.h), args.cmp_steps, 3,
+                               torch)
+        t_unf_up = time_loop(layer.unfused_up, args.cmp_steps, 3, torch)
+        result["unfused"] = {
+            "qkv": {"fused_us": t_fused_qkv * 1e3, "unfused_us": t_unf_qkv * 1e3,
+                    "speedup": t_unf_qkv / t_fused_qkv},
+            "ffn_up": {"fused_us": t_fused_up * 1e3, "unfused_us": t_unf_up * 1e3,
+                       "speedup": t_unf_up / t_fused_up},
+            "note": "unfused = plain NVFP4 GEMM writing bf16, then rmsnorm_heads_bf16 (in place) / "
+                    "swiglu_bf16 + nvfp4_quantize (static scale); same kernels' library",
+        }
+        del layer.c_up, layer.y_up
+        torch.cuda.empty_cache()
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        x_host = layer.x.cpu().pin_memory()
+        qkv_host = torch.empty(layer.qkv.shape, dtype=torch.bfloat16).pin_memory()
+        out_host = torch.empty(layer.out.shape, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            layer.x.copy_(x_host, non_blocking=True)
+            layer.step()
+            qkv_host.copy_(layer.qkv, non_blocking=True)
+            out_host.copy_(layer.out, non_blocking=True)
+
+        barrier()
+        t_e2e = time_loop(e2e_step, max(2, K // 2), 2, torch)
+        te = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        t_e2e = float(te.item())
+        result["e2e"] = {"value": round(total_flops * world / (t_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                         "h2d_bytes_per_step": int(x_host.numel() * 2),
+                         "d2h_bytes_per_step": int((qkv_host.numel() + out_host.numel()) * 2),
+                         "ms_per_step": round(t_e2e, 4)}
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(M, rows=args.cpu_rows)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+# ----------------------------------------------------------------------------------
+# the CPU oracle arm
+# ----------------------------------------------------------------------------------
+class OracleLayer:
+    """The oracle's pieces of the same step; weight packing done once (model load)."""
+
+    def __init__(self, M: int, seed: int = 0):
+        from oracle import nvfp4_oracle as o
+        import workloads as wk
+        self.o = o
+        self.M = M
+        self.x = wk.activations(M, K_IN, wk.outlier_count(K_IN), seed=seed).float().numpy()
+        std = 1.0 / np.sqrt(K_IN)
+        t0 = time.perf_counter()
+        self.Bqkv = o.dequantize(*o.quantize(wk.weights(N_QKV, K_IN, std, seed=seed, stream=11).float().numpy()))
+        self.Bup = o.dequantize(*o.quantize(wk.weights(N_UP, K_IN, std, seed=seed, stream=12).float().numpy()))
+        self.Bdown = o.dequantize(*o.quantize(
+            wk.weights(K_IN, K_DOWN, 1.0 / np.sqrt(K_DOWN), seed=seed, stream=13).float().numpy()))
+        self.pack_s = time.perf_counter() - t0
+        wq, wkk = wk.norm_weight(HD, seed, 3), wk.norm_weight(HD, seed, 5)
+        self.w = np.concatenate([np.tile(wq, N_NORM // 2 // HD), np.tile(wkk, N_NORM // 2 // HD)])
+        self.Gx = o.global_scale(self.x)
+        self.Gh = None
+
+    def step(self, rows):
+        o = self.o
+        xs = self.x[rows]
+        qa, sa, _ = o.quantize(xs, self.Gx)
+        a = o.dequantize(qa, sa, self.Gx)
+        qkv = o.bf16_round(o.rmsnorm_heads(o.gemm(a, self.Bqkv), self.w, HD, N_NORM, EPS))
+        h = o.bf16_round(o.swiglu(o.gemm(a, self.Bup)))
+        if self.Gh is None:
+            self.Gh = np.float32(np.abs(h).max() / 2688)
+        qh, sh, _ = o.requantize(h, self.Gh)
+        out = o.bf16_round(o.gemm(o.dequantize(qh, sh, self.Gh), self.Bdown))
+        return qkv, out
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:  # pragma: no cover
+        return os.cpu_count()
+
+
+def cpu_baseline(M: int, rows: int = 256):
+    layer = OracleLayer(M)
+    rng = np.random.default_rng(0)
+    sample = np.sort(rng.choice(M, size=rows, replace=False))
+    t0 = time.perf_counter()
+    layer.step(sample)
+    dt = time.perf_counter() - t0
+    fl = sum(step_flops(rows).values())
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{rows} random rows of the M={M} step (quantise, fp64 GEMMs, RMSNorm, SwiGLU, requant, "
+                      f"down GEMM) in {dt:.2f} s; weight packing ({layer.pack_s:.1f} s, once per model) excluded",
+            "host_threads": os.cpu_count()}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    layer = OracleLayer(args.M)
+    rng = np.random.default_rng(1)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        layer.step(np.sort(rng.choice(args.M, size=rows, replace=False)))
+    t = 0.0
+    for _ in range(args.steps):
+        sample = np.sort(rng.choice(args.M, size=rows, replace=False))
+        t0 = time.perf_counter()
+        layer.step(sample)
+        t += time.perf_counter() - t0
+    fl = sum(step_flops(rows).values())
+    value = fl * args.steps / t / 1e12
+    cores = _blas_threads()
+    out = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": workload_desc(args.M), "M": args.M,
+                      "sample_rows_per_step": rows, "parallelism": "cpu oracle, rank 0 only"},
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                            "sample": f"{rows} random rows of the M={args.M} step per step; weight packing "
+                                      f"({layer.pack_s:.1f} s) done once before timing"},
+           "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--M", type=int, default=16384, help="tokens per GPU per step")
+    ap.add_argument("--cmp-steps", type=int, default=10, help="steps of each fused/unfused comparison loop")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="rows of the oracle sample in cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=64, help="rows per step of the --impl reference arm")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the FFN-up kernel from an ncu capture of this kernel")
+    ap.add_argument("--no-unfused", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()
