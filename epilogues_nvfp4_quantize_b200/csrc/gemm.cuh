@@ -4,28 +4,31 @@
 // in brief": the tensor cores accumulate a tile in TMEM while HBM is not touched for the
 // output; the small op is applied to the accumulator and the result is written once.
 //
-// Structure (one persistent CTA per SM, 320 threads, warp-specialised):
-//   warp 8     TMA producer: A/B code tiles (128-byte swizzle) and their scale units,
-//              3-stage shared-memory ring, one mbarrier pair per stage;
-//   warp 9     TMEM owner and MMA issuer: copies the stage's E4M3 scales into TMEM
-//              (tcgen05.cp) and issues 4 block-scaled MMAs of 128 x 256 x 64 per stage;
-//   warps 0-7  epilogue: warp w reads TMEM lanes 32*(w%4).. (its 32 output rows) and
-//              columns 128*(w/4).. (its half of the 256-column tile); each thread owns one
-//              output row. Results go through a swizzled staging box and a TMA store.
-// Tile = 128 x 256 outputs, K step = 256 (one 128-byte swizzle row of FP4 codes).
+// Two kernels share the epilogue:
+//   gemm_nvfp4_pair_kernel  (M % 256 == 0) a cluster of 2 CTAs on the two SMs of a TPC
+//       runs one 256 x 256 output tile with the pair MMA (tcgen05 cta_group::2): each CTA
+//       stages its own 128 rows of A and 128 of the 256 rows of B, so a CTA moves
+//       38 KB per K step of 256 for 128 x 256 x 256 MMA work (5-stage ring);
+//   gemm_nvfp4_kernel       (M % 256 == 128) one CTA per 128 x 256 tile (3-stage ring).
+// Warp roles (320 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
+// and MMA issuer. Epilogue warp w reads TMEM lanes 32*(w%4).. (its 32 output rows) and
+// columns 128*(w/4).. (its half of the 256-column tile); each thread owns one output row.
+// Results go through a 128-byte-swizzled staging box and a TMA store.
 //
 // Epilogues:
-//   PLAIN    y = alpha * acc
+//   PLAIN    y = alpha * acc,  alpha = G_A * G_B
 //   RMSNORM  per head of 128 or 256 columns (sections "Tiles and fragments on Blackwell",
-//            "Why head_dim=256 is hard", "Revisit fusion"): first touch accumulates the
-//            sum of squares of the thread's 128 columns; a 256-wide head spans the two
-//            epilogue warpgroups, which exchange their partial sums through shared memory
-//            (an mbarrier, so the wait stays bounded); second touch re-reads TMEM,
-//            scales by rstd * w and stores. Columns past n_norm_cols pass through.
+//            "Why head_dim=256 is hard", "Revisit fusion"): a first touch of TMEM
+//            accumulates the sum of squares of the thread's 128 columns; a 256-wide head
+//            spans the two epilogue warpgroups, which exchange their partial sums through
+//            shared memory (an mbarrier, so the wait stays bounded); a second touch
+//            re-reads TMEM, scales by rstd * w and stores. Columns past n_norm_cols pass
+//            through.
 //   SWIGLU   accumulator columns come interleaved [g0, u0, g1, u1, ...] from the weight
 //            packing of section "Fusing gated SiLU (SwiGLU)", so each thread computes
-//            silu(g) * u on adjacent columns of its own row; optional NVFP4 re-quantisation
-//            of the bf16-rounded result with a static scale, 16 outputs per block.
+//            silu(g) * u on adjacent columns of its own row; optional NVFP4
+//            re-quantisation of the bf16-rounded result with a static scale, one 16-block
+//            per 32 accumulator columns.
 #pragma once
 
 #include "ptx.cuh"
@@ -37,34 +40,41 @@ namespace nvfp4 {
 enum EpiKind { EPI_PLAIN = 0, EPI_RMSNORM = 1, EPI_SWIGLU = 2 };
 
 namespace gemm_cfg {
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                 // output rows per CTA
+constexpr int BN = 256;                 // output columns per tile
 constexpr int BK = 256;                 // FP4 elements per stage along K
-constexpr int BK_BYTES = BK / 2;        // 128
-constexpr int STAGES = 3;
-constexpr int A_BYTES = BM * BK_BYTES;  // 16 KB
-constexpr int B_BYTES = BN * BK_BYTES;  // 32 KB
+constexpr int BK_BYTES = BK / 2;        // 128: one swizzle row
 constexpr int SF_UNIT = 512;            // scales of 128 rows x 64 K
-constexpr int SFA_BYTES = (BM / 128) * (BK / 64) * SF_UNIT;  // 2 KB
-constexpr int SFB_BYTES = (BN / 128) * (BK / 64) * SF_UNIT;  // 4 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
 constexpr int NUM_THREADS = EPI_THREADS + 64;
 constexpr int BOX_BYTES = 32 * 128;     // one staging box: 32 rows x 128 bytes
-constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-constexpr int OFF_RED = OFF_EPI + EPI_WARPS * BOX_BYTES;
-constexpr int OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
-constexpr int NUM_BARS = 2 * STAGES + 4;
-constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+constexpr int RED_BYTES = 2 * 2 * 128 * 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;    // 256 fp32 columns
 constexpr uint32_t SFA_COL = 256;  // 4 MMAs x 4 columns
 constexpr uint32_t SFB_COL = 272;  // 4 MMAs x 8 columns
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace gemm_cfg
+
+// Shared-memory plan of a kernel with S stages of B_ROWS rows of B per CTA.
+template <int S, int B_ROWS>
+struct SmemPlan {
+  static constexpr int A_BYTES = gemm_cfg::BM * gemm_cfg::BK_BYTES;                 // 16 KB
+  static constexpr int B_BYTES = B_ROWS * gemm_cfg::BK_BYTES;                       // 16 or 32 KB
+  static constexpr int SFA_BYTES = (gemm_cfg::BK / 64) * gemm_cfg::SF_UNIT;          // 2 KB
+  static constexpr int SFB_BYTES = 2 * (gemm_cfg::BK / 64) * gemm_cfg::SF_UNIT;      // 4 KB (256 rows)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int OFF_EPI = S * STAGE_BYTES;
+  static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
+  static constexpr int OFF_BAR = OFF_RED + gemm_cfg::RED_BYTES;
+  static constexpr int NUM_BARS = 2 * S + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+using PlanSingle = SmemPlan<3, 256>;
+using PlanPair = SmemPlan<5, 128>;
 
 struct GemmArgs {
   const uint8_t* sfa;
@@ -72,7 +82,8 @@ struct GemmArgs {
   const float* ga;
   const float* gb;
   int M, N, K;
-  int tiles_m, tiles_n, num_tiles;
+  int tiles_m, tiles_n, num_tiles;  // in units of the kernel's tile (128 or 256 rows)
+  int n_fastest;                    // tile order: 1 = N index fastest (B stays in L2)
   // RMSNorm
   const float* w;
   int head_dim;
@@ -86,6 +97,16 @@ struct GemmArgs {
   int q_cols;           // Nh
   uint64_t wait_limit_ns;
 };
+
+__device__ __forceinline__ void tile_coords(const GemmArgs& a, int t, int& tm, int& tn) {
+  if (a.n_fastest) {
+    tn = t % a.tiles_n;
+    tm = t / a.tiles_n;
+  } else {
+    tm = t % a.tiles_m;
+    tn = t / a.tiles_m;
+  }
+}
 
 // Write 64 bf16 values (32 packed words) of this thread's row into the 128-byte-swizzled
 // staging box (32 rows x 128 bytes); chunk q of row i goes to chunk q ^ (i % 8).
@@ -113,22 +134,199 @@ __device__ __forceinline__ void box_reuse_wait(int lane) {
   __syncwarp();
 }
 
+// Per-warp state of the epilogue.
+struct EpiCtx {
+  const GemmArgs* args;
+  const CUtensorMap* tmD;
+  uint32_t t_row;     // TMEM address of lane 32*sub, column 0
+  int wg, sub, lane;
+  uint8_t* box;
+  float* red;
+  uint64_t* red_bar;
+  uint32_t xchg;
+  volatile int* abort_flag;
+  float alpha, qG, qenc;
+};
+
+// Epilogue of one tile: this CTA's 128 rows starting at m0, 256 accumulator columns
+// starting at n0. `release()` is called by every thread once its last TMEM read of the
+// tile has completed (the accumulator may then be overwritten). Returns false if a
+// bounded wait gave up.
+template <int EPI, class Release>
+__device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release release) {
+  using namespace gemm_cfg;
+  const GemmArgs& args = *c.args;
+  const int lane = c.lane;
+  const uint32_t tcol = c.t_row + ACC_COL + c.wg * 128;
+  const int col0 = n0 + c.wg * 128;
+  const int row_in_tile = c.sub * 32 + lane;
+  const float alpha = c.alpha;
+
+  if constexpr (EPI == EPI_SWIGLU) {
+    uint32_t packed[32];
+    uint32_t qc[8];
+    uint32_t sfw = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v[32];
+      tmem_ld32(tcol + 32 * q, v);
+      tmem_ld_wait();
+      if (q == 3) release();
+      float o[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float g = alpha * __uint_as_float(v[2 * j]);
+        const float u = alpha * __uint_as_float(v[2 * j + 1]);
+        o[j] = silu_f32(g) * u;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) packed[8 * q + j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
+      if (args.q_codes != nullptr) {
+        float ob[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          ob[2 * j] = bf16_lo(packed[8 * q + j]);
+          ob[2 * j + 1] = bf16_hi(packed[8 * q + j]);
+        }
+        uint32_t lo, hi;
+        const uint32_t s = quant_block16(ob, c.qG, c.qenc, lo, hi);
+        qc[2 * q] = lo;
+        qc[2 * q + 1] = hi;
+        sfw |= s << (8 * q);
+      }
+    }
+    const int oc0 = col0 >> 1;  // first of this thread's 64 output columns
+    if (args.write_d) {
+      box_reuse_wait(lane);
+      stage_row_bf16(c.box, lane, packed);
+      flush_box(c.tmD, c.box, lane, oc0, m0 + c.sub * 32);
+    }
+    if (args.q_codes != nullptr) {
+      const int64_t row = m0 + row_in_tile;
+      uint4* dst = reinterpret_cast<uint4*>(args.q_codes + row * (args.q_cols >> 1) + (oc0 >> 1));
+      dst[0] = make_uint4(qc[0], qc[1], qc[2], qc[3]);
+      dst[1] = make_uint4(qc[4], qc[5], qc[6], qc[7]);
+      *reinterpret_cast<uint32_t*>(args.q_sf + sf_word_offset(row, oc0 >> 4, args.q_cols >> 4)) = sfw;
+    }
+    return true;
+  } else {
+    // PLAIN, or RMSNORM (normalised half) / its passthrough half
+    bool norm = false;
+    float rstd = 1.0f;
+    if constexpr (EPI == EPI_RMSNORM) {
+      norm = col0 < args.n_norm_cols;
+      if (norm) {
+        float ss = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; q += 2) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tcol + 32 * q, v0);
+          tmem_ld32(tcol + 32 * q + 32, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float a = alpha * __uint_as_float(v0[j]);
+            const float b = alpha * __uint_as_float(v1[j]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+        float mean;
+        if (args.head_dim == 256) {
+          float* slot = c.red + (c.xchg & 1u) * 256;
+          slot[c.wg * 128 + row_in_tile] = ss;
+          mbar_arrive(c.red_bar);
+          if (!__all_sync(0xffffffffu, mbar_wait(c.red_bar, c.xchg & 1u, c.abort_flag, args.wait_limit_ns, 5)))
+            return false;
+          ss = slot[row_in_tile] + slot[128 + row_in_tile];
+          ++c.xchg;
+          mean = ss * (1.0f / 256.0f);
+        } else {
+          mean = ss * (1.0f / 128.0f);
+        }
+        rstd = rsqrtf(mean + args.eps);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tcol + 64 * h, v0);
+      tmem_ld32(tcol + 64 * h + 32, v1);
+      tmem_ld_wait();
+      if (h == 1) release();
+      uint32_t p[32];
+      if (EPI == EPI_RMSNORM && norm) {
+        const float* wp = args.w + col0 + 64 * h;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float2 wa = __ldg(reinterpret_cast<const float2*>(wp + 2 * j));
+          const float2 wb = __ldg(reinterpret_cast<const float2*>(wp + 32 + 2 * j));
+          p[j] = pack_bf16x2(alpha * __uint_as_float(v0[2 * j]) * rstd * wa.x,
+                             alpha * __uint_as_float(v0[2 * j + 1]) * rstd * wa.y);
+          p[16 + j] = pack_bf16x2(alpha * __uint_as_float(v1[2 * j]) * rstd * wb.x,
+                                  alpha * __uint_as_float(v1[2 * j + 1]) * rstd * wb.y);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          p[j] = pack_bf16x2(alpha * __uint_as_float(v0[2 * j]), alpha * __uint_as_float(v0[2 * j + 1]));
+          p[16 + j] = pack_bf16x2(alpha * __uint_as_float(v1[2 * j]), alpha * __uint_as_float(v1[2 * j + 1]));
+        }
+      }
+      box_reuse_wait(lane);
+      stage_row_bf16(c.box, lane, p);
+      flush_box(c.tmD, c.box, lane, col0 + 64 * h, m0 + c.sub * 32);
+    }
+    return true;
+  }
+}
+
+__device__ __forceinline__ EpiCtx make_epi_ctx(const GemmArgs& args, const CUtensorMap* tmD, uint32_t tmem,
+                                               uint8_t* smem, int off_epi, int off_red, uint64_t* red_bar,
+                                               volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5;
+  EpiCtx c;
+  c.args = &args;
+  c.tmD = tmD;
+  c.wg = warp >> 2;
+  c.sub = warp & 3;
+  c.lane = threadIdx.x & 31;
+  c.t_row = tmem + (static_cast<uint32_t>(c.sub * 32) << 16);
+  c.box = smem + off_epi + warp * gemm_cfg::BOX_BYTES;
+  c.red = reinterpret_cast<float*>(smem + off_red);
+  c.red_bar = red_bar;
+  c.xchg = 0;
+  c.abort_flag = abort_flag;
+  c.alpha = __fmul_rn(*args.ga, *args.gb);
+  c.qG = 0.0f;
+  c.qenc = 0.0f;
+  if (args.q_codes != nullptr) {
+    c.qG = *args.q_gscale;
+    c.qenc = scale_encode_factor(c.qG);
+  }
+  return c;
+}
+
+// =====================================================================================
+// One CTA per 128 x 256 tile (used when M % 256 == 128)
+// =====================================================================================
 template <int EPI>
 __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
   using namespace gemm_cfg;
+  using P = PlanSingle;
+  constexpr int STAGES = 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* red_bar = acc_full + 2;
   uint64_t* drain_bar = acc_full + 3;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
-  float* red = reinterpret_cast<float*>(smem + OFF_RED);  // [2 parity][2 wg][128 rows]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -140,7 +338,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, EPI_THREADS);
+    mbar_init(acc_empty, EPI_WARPS);
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -171,22 +369,24 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
       int issued = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
-        const int tm = t % args.tiles_m, tn = t / args.tiles_m;
+        int tm, tn;
+        tile_coords(args, t, tm, tn);
         for (int kt = 0; kt < ktiles; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 1)) {
             ok = false;
             break;
           }
-          uint8_t* sb = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          uint8_t* sb = smem + stage * P::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], P::STAGE_BYTES);
           tma_load_2d(sb, &tmA, &full[stage], kt * BK_BYTES, tm * BM);
-          tma_load_2d(sb + A_BYTES, &tmB, &full[stage], kt * BK_BYTES, tn * BN);
+          tma_load_2d(sb + P::A_BYTES, &tmB, &full[stage], kt * BK_BYTES, tn * BN);
           const int64_t ka = static_cast<int64_t>(kt) * (BK / 64);
-          bulk_load(sb + A_BYTES + B_BYTES, args.sfa + (tm * kunits + ka) * SF_UNIT, SFA_BYTES, &full[stage]);
-          bulk_load(sb + A_BYTES + B_BYTES + SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT,
-                    SFB_BYTES / 2, &full[stage]);
-          bulk_load(sb + A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES / 2,
-                    args.sfb + ((2 * tn + 1) * kunits + ka) * SF_UNIT, SFB_BYTES / 2, &full[stage]);
+          uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
+          bulk_load(ssf, args.sfa + (tm * kunits + ka) * SF_UNIT, P::SFA_BYTES, &full[stage]);
+          bulk_load(ssf + P::SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT, P::SFB_BYTES / 2,
+                    &full[stage]);
+          bulk_load(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, args.sfb + ((2 * tn + 1) * kunits + ka) * SF_UNIT,
+                    P::SFB_BYTES / 2, &full[stage]);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -194,7 +394,17 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
+      if (ok) {
+        // Tail: wait until the MMAs have released every stage still in use, so that no
+        // arrival reaches this CTA's barriers after it exits.
+        for (int i = 0; i < STAGES && i < issued; ++i) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 13)) break;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      } else {
         // Give up: wait (bounded) for the copies this thread started, then leave.
         for (int i = 0; i < STAGES && i < issued; ++i) {
           if (--stage < 0) {
@@ -224,15 +434,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t b_addr = a_addr + A_BYTES;
-          const uint32_t sfa_addr = b_addr + B_BYTES;
-          const uint32_t sfb_addr = sfa_addr + SFA_BYTES;
+          const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + P::A_BYTES;
+          const uint32_t sfa_addr = b_addr + P::B_BYTES;
+          const uint32_t sfb_addr = sfa_addr + P::SFA_BYTES;
 #pragma unroll
           for (int j = 0; j < BK / 64; ++j) {
             tc_copy_scales(tmem + SFA_COL + 4 * j, smem_desc_scales(sfa_addr + j * SF_UNIT));
             tc_copy_scales(tmem + SFB_COL + 8 * j, smem_desc_scales(sfb_addr + j * SF_UNIT));
-            tc_copy_scales(tmem + SFB_COL + 8 * j + 4, smem_desc_scales(sfb_addr + SFB_BYTES / 2 + j * SF_UNIT));
+            tc_copy_scales(tmem + SFB_COL + 8 * j + 4, smem_desc_scales(sfb_addr + P::SFB_BYTES / 2 + j * SF_UNIT));
           }
           const uint64_t adesc = smem_desc_sw128(a_addr);
           const uint64_t bdesc = smem_desc_sw128(b_addr);
@@ -259,147 +469,20 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int wg = warp >> 2;          // column half of the tile
-    const int sub = warp & 3;          // TMEM lane quadrant = output row group
-    const int row_in_tile = sub * 32 + lane;
-    uint8_t* box = smem + OFF_EPI + warp * BOX_BYTES;
-    const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-    const float alpha = __fmul_rn(*args.ga, *args.gb);
-    float qG = 0.0f, qenc = 0.0f;
-    if (EPI == EPI_SWIGLU && args.q_codes != nullptr) {
-      qG = *args.q_gscale;
-      qenc = scale_encode_factor(qG);
-    }
-    uint32_t acc_phase = 0, xchg = 0;
+    EpiCtx c = make_epi_ctx(args, &tmD, tmem, smem, P::OFF_EPI, P::OFF_RED, red_bar, abort_flag);
+    auto release = [&]() {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+    };
+    uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
-      const int tm = t % args.tiles_m, tn = t / args.tiles_m;
-      const int m0 = tm * BM, n0 = tn * BN;
+      int tm, tn;
+      tile_coords(args, t, tm, tn);
       // every lane waits; the warp leaves together if any lane gave up
       if (!__all_sync(0xffffffffu, mbar_wait(acc_full, acc_phase, abort_flag, limit, 4))) break;
       tc_fence_after();
-      const uint32_t tcol = t_row + ACC_COL + wg * 128;
-      const int col0 = n0 + wg * 128;
-
-      if constexpr (EPI == EPI_SWIGLU) {
-        uint32_t packed[32];
-        uint32_t qc[8];
-        uint32_t sfw = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t v[32];
-          tmem_ld32(tcol + 32 * q, v);
-          tmem_ld_wait();
-          if (q == 3) {
-            tc_fence_before();
-            mbar_arrive(acc_empty);
-          }
-          float o[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float g = alpha * __uint_as_float(v[2 * j]);
-            const float u = alpha * __uint_as_float(v[2 * j + 1]);
-            o[j] = silu_f32(g) * u;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) packed[8 * q + j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
-          if (args.q_codes != nullptr) {
-            float ob[16];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              ob[2 * j] = bf16_lo(packed[8 * q + j]);
-              ob[2 * j + 1] = bf16_hi(packed[8 * q + j]);
-            }
-            uint32_t lo, hi;
-            const uint32_t s = quant_block16(ob, qG, qenc, lo, hi);
-            qc[2 * q] = lo;
-            qc[2 * q + 1] = hi;
-            sfw |= s << (8 * q);
-          }
-        }
-        const int oc0 = col0 >> 1;  // first of this thread's 64 output columns
-        if (args.write_d) {
-          box_reuse_wait(lane);
-          stage_row_bf16(box, lane, packed);
-          flush_box(&tmD, box, lane, oc0, m0 + sub * 32);
-        }
-        if (args.q_codes != nullptr) {
-          const int64_t row = m0 + row_in_tile;
-          uint4* dst = reinterpret_cast<uint4*>(args.q_codes + row * (args.q_cols >> 1) + (oc0 >> 1));
-          dst[0] = make_uint4(qc[0], qc[1], qc[2], qc[3]);
-          dst[1] = make_uint4(qc[4], qc[5], qc[6], qc[7]);
-          *reinterpret_cast<uint32_t*>(args.q_sf + sf_word_offset(row, oc0 >> 4, args.q_cols >> 4)) = sfw;
-        }
-      } else {
-        // PLAIN, or RMSNORM (normalised half) / its passthrough half
-        bool norm = false;
-        float rstd = 1.0f;
-        if constexpr (EPI == EPI_RMSNORM) {
-          norm = col0 < args.n_norm_cols;
-          if (norm) {
-            float ss = 0.0f;
-#pragma unroll
-            for (int q = 0; q < 4; q += 2) {
-              uint32_t v0[32], v1[32];
-              tmem_ld32(tcol + 32 * q, v0);
-              tmem_ld32(tcol + 32 * q + 32, v1);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float a = alpha * __uint_as_float(v0[j]);
-                const float b = alpha * __uint_as_float(v1[j]);
-                ss = fmaf(a, a, ss);
-                ss = fmaf(b, b, ss);
-              }
-            }
-            float mean;
-            if (args.head_dim == 256) {
-              float* slot = red + (xchg & 1u) * 256;
-              slot[wg * 128 + row_in_tile] = ss;
-              mbar_arrive(red_bar);
-              if (!__all_sync(0xffffffffu, mbar_wait(red_bar, xchg & 1u, abort_flag, limit, 5))) break;
-              ss = slot[row_in_tile] + slot[128 + row_in_tile];
-              ++xchg;
-              mean = ss * (1.0f / 256.0f);
-            } else {
-              mean = ss * (1.0f / 128.0f);
-            }
-            rstd = rsqrtf(mean + args.eps);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tcol + 64 * h, v0);
-          tmem_ld32(tcol + 64 * h + 32, v1);
-          tmem_ld_wait();
-          if (h == 1) {
-            tc_fence_before();
-            mbar_arrive(acc_empty);
-          }
-          uint32_t p[32];
-          if (EPI == EPI_RMSNORM && norm) {
-            const float* wp = args.w + col0 + 64 * h;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float2 wa = __ldg(reinterpret_cast<const float2*>(wp + 2 * j));
-              const float2 wb = __ldg(reinterpret_cast<const float2*>(wp + 32 + 2 * j));
-              p[j] = pack_bf16x2(alpha * __uint_as_float(v0[2 * j]) * rstd * wa.x,
-                                 alpha * __uint_as_float(v0[2 * j + 1]) * rstd * wa.y);
-              p[16 + j] = pack_bf16x2(alpha * __uint_as_float(v1[2 * j]) * rstd * wb.x,
-                                      alpha * __uint_as_float(v1[2 * j + 1]) * rstd * wb.y);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              p[j] = pack_bf16x2(alpha * __uint_as_float(v0[2 * j]), alpha * __uint_as_float(v0[2 * j + 1]));
-              p[16 + j] = pack_bf16x2(alpha * __uint_as_float(v1[2 * j]), alpha * __uint_as_float(v1[2 * j + 1]));
-            }
-          }
-          box_reuse_wait(lane);
-          stage_row_bf16(box, lane, p);
-          flush_box(&tmD, box, lane, col0 + 64 * h, m0 + sub * 32);
-        }
-      }
+      if (!epilogue_tile<EPI>(c, tm * BM, tn * BN, release)) break;
       acc_phase ^= 1u;
     }
     if (lane == 0) bulk_wait_all();
@@ -411,6 +494,208 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   if (warp == EPI_WARPS + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// =====================================================================================
+// A CTA pair per 256 x 256 tile (used when M % 256 == 0). Cluster of 2 CTAs; CTA rank r
+// owns output rows [m0 + 128 r, m0 + 128 r + 128) and stages B rows [n0 + 128 r, +128).
+// =====================================================================================
+template <int EPI>
+__global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
+    gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                           const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
+  using namespace gemm_cfg;
+  using P = PlanPair;
+  constexpr int STAGES = 5;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* red_bar = acc_full + 2;
+  uint64_t* drain_bar = acc_full + 3;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t limit = args.wait_limit_ns;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // leader's: one expect-tx arrival, both CTAs' bytes
+      mbar_init(&empty[s], 1);  // one multicast commit per use
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * EPI_WARPS);  // leader's: one arrival per epilogue warp of the pair
+    mbar_init(red_bar, EPI_THREADS);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == EPI_WARPS && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmSFA);
+    prefetch_tensormap(&tmSFB);
+    if (args.write_d) prefetch_tensormap(&tmD);
+  }
+  // barrier inits visible cluster-wide before any remote arrival or pair allocation
+  cluster_sync_all();
+  if (warp == EPI_WARPS + 1) {
+    tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int ktiles = args.K / BK;
+  const int kunits = args.K / 64;
+
+  if (warp == EPI_WARPS) {
+    // ------------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters) {
+        int tm, tn;
+        tile_coords(args, t, tm, tn);
+        const int a_row = tm * 256 + 128 * static_cast<int>(rank);   // this CTA's A rows
+        const int b_row = tn * 256 + 128 * static_cast<int>(rank);   // this CTA's half of B
+        const int sfa_group = a_row / 128;
+        for (int kt = 0; kt < ktiles; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 21)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = smem + stage * P::STAGE_BYTES;
+          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P::STAGE_BYTES);
+          tma_load_2d_pair(sb, &tmA, bar, kt * BK_BYTES, a_row);
+          tma_load_2d_pair(sb + P::A_BYTES, &tmB, bar, kt * BK_BYTES, b_row);
+          // scale units: 512 bytes = 2 rows of the 256-byte-wide scale tensor map
+          uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
+          tma_load_2d_pair(ssf, &tmSFA, bar, 0, 2 * (sfa_group * kunits + 4 * kt));
+          tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar, 0, 2 * ((2 * tn) * kunits + 4 * kt));
+          tma_load_2d_pair(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, &tmSFB, bar, 0,
+                           2 * ((2 * tn + 1) * kunits + 4 * kt));
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (ok) {
+        for (int i = 0; i < STAGES && i < issued; ++i) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 23)) break;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      } else if (leader) {
+        // both CTAs' copies complete on the leader's barriers: wait (bounded) for them
+        for (int i = 0; i < STAGES && i < issued; ++i) {
+          if (--stage < 0) {
+            stage = STAGES - 1;
+            phase ^= 1u;
+          }
+          (void)mbar_wait(&full[stage], phase, nullptr, limit, 24);
+        }
+      }
+    }
+  } else if (warp == EPI_WARPS + 1) {
+    // ------------------------------------------------------------------ MMA issuer (leader only)
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_nvfp4(2 * BM, BN);
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, limit, 22)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < ktiles; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + P::A_BYTES;
+          const uint32_t sfa_addr = b_addr + P::B_BYTES;
+          const uint32_t sfb_addr = sfa_addr + P::SFA_BYTES;
+#pragma unroll
+          for (int j = 0; j < BK / 64; ++j) {
+            tc_copy_scales_pair(tmem + SFA_COL + 4 * j, smem_desc_scales(sfa_addr + j * SF_UNIT));
+            tc_copy_scales_pair(tmem + SFB_COL + 8 * j, smem_desc_scales(sfb_addr + j * SF_UNIT));
+            tc_copy_scales_pair(tmem + SFB_COL + 8 * j + 4,
+                                smem_desc_scales(sfb_addr + P::SFB_BYTES / 2 + j * SF_UNIT));
+          }
+          const uint64_t adesc = smem_desc_sw128(a_addr);
+          const uint64_t bdesc = smem_desc_sw128(b_addr);
+#pragma unroll
+          for (int kb = 0; kb < BK / 64; ++kb) {
+            tc_mma_nvfp4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
+                              tmem + SFB_COL + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(acc_full, 0x3);
+        acc_phase ^= 1u;
+      }
+      if (!ok) {
+        tc_commit_pair(drain_bar, 0x1);
+        (void)mbar_wait(drain_bar, 0, nullptr, limit, 26);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    EpiCtx c = make_epi_ctx(args, &tmD, tmem, smem, P::OFF_EPI, P::OFF_RED, red_bar, abort_flag);
+    const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
+    auto release = [&]() {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
+    };
+    uint32_t acc_phase = 0;
+    for (int t = cluster_id; t < args.num_tiles; t += num_clusters) {
+      int tm, tn;
+      tile_coords(args, t, tm, tn);
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full, acc_phase, abort_flag, limit, 27))) break;
+      tc_fence_after();
+      if (!epilogue_tile<EPI>(c, tm * 256 + 128 * static_cast<int>(rank), tn * BN, release)) break;
+      acc_phase ^= 1u;
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  // both CTAs done with each other's barriers and with the pair's TMEM
+  cluster_sync_all();
+  if (warp == EPI_WARPS + 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 

@@ -31,6 +31,8 @@ struct DeviceInfo {
   bool supported = false;
   int sm_count = 0;
   bool gemm_attr_set[3] = {false, false, false};
+  bool pair_attr_set[3] = {false, false, false};
+  int pair_clusters[3] = {0, 0, 0};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -78,7 +80,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -86,7 +88,7 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -97,7 +99,8 @@ nvfp4_status check_operand(const nvfp4_tensor& t) {
   return NVFP4_OK;
 }
 
-// Common checks and launch of the GEMM kernel template.
+// Common checks and launch of the GEMM kernels: the CTA-pair kernel when M % 256 == 0,
+// the single-CTA kernel otherwise.
 template <int EPI>
 nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int64_t ldd, int64_t n_out,
                       nvfp4::GemmArgs args, cudaStream_t stream) {
@@ -117,13 +120,24 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   DeviceInfo* info;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
 
-  CUtensorMap tmA, tmB, tmD;
+  const bool pair = (M % 256) == 0;
+  CUtensorMap tmA, tmB, tmD, tmSFA, tmSFB;
   std::memset(&tmD, 0, sizeof(tmD));
-  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.codes, K / 2, M, K / 2, BK_BYTES, BM) ||
-      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B.codes, K / 2, N, K / 2, BK_BYTES, BN))
+  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.codes, K / 2, M, K / 2, BK_BYTES, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B.codes, K / 2, N, K / 2, BK_BYTES, pair ? 128 : BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ERR_CUDA;
+  if (pair) {
+    // the block scales seen as rows of 256 bytes; one 128-row x 256-K group = 8 rows
+    if (!make_map_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.sf, 256, M * (K / 16) / 256, 256, 256, 8,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B.sf, 256, N * (K / 16) / 256, 256, 256, 8,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return NVFP4_ERR_CUDA;
+  }
   if (D != nullptr &&
-      !make_map_2d(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, n_out, M, ldd * 2, 64, 32))
+      !make_map_2d(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, n_out, M, ldd * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ERR_CUDA;
 
   args.sfa = static_cast<const uint8_t*>(A.sf);
@@ -133,23 +147,62 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   args.M = static_cast<int>(M);
   args.N = static_cast<int>(N);
   args.K = static_cast<int>(K);
-  args.tiles_m = static_cast<int>(M / BM);
+  args.tiles_m = static_cast<int>(M / (pair ? 256 : BM));
   args.tiles_n = static_cast<int>(N / BN);
   args.num_tiles = args.tiles_m * args.tiles_n;
+  // keep the smaller operand resident in L2 while the larger one streams through once
+  args.n_fastest = N <= M ? 1 : 0;
   args.write_d = D != nullptr;
   args.wait_limit_ns = kWaitLimitNs;
 
-  auto kern = nvfp4::gemm_nvfp4_kernel<EPI>;
+  if (!pair) {
+    using P = nvfp4::PlanSingle;
+    auto kern = nvfp4::gemm_nvfp4_kernel<EPI>;
+    {
+      std::lock_guard<std::mutex> lock(g_mutex);
+      if (!info->gemm_attr_set[EPI]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
+          return NVFP4_ERR_CUDA;
+        info->gemm_attr_set[EPI] = true;
+      }
+    }
+    const int grid = args.num_tiles < info->sm_count ? args.num_tiles : info->sm_count;
+    kern<<<grid, NUM_THREADS, P::SMEM_BYTES, stream>>>(tmA, tmB, tmD, args);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return launch_status();
+  }
+
+  using P = nvfp4::PlanPair;
+  auto kern = nvfp4::gemm_nvfp4_pair_kernel<EPI>;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = P::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_clusters;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!info->gemm_attr_set[EPI]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    if (!info->pair_attr_set[EPI]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
         return NVFP4_ERR_CUDA;
-      info->gemm_attr_set[EPI] = true;
+      cfg.gridDim = dim3(2 * (info->sm_count / 2), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return NVFP4_ERR_CUDA;
+      info->pair_clusters[EPI] = n;
+      info->pair_attr_set[EPI] = true;
     }
+    max_clusters = info->pair_clusters[EPI];
   }
-  const int grid = static_cast<int>(args.num_tiles < info->sm_count ? args.num_tiles : info->sm_count);
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmD, args);
+  const int clusters = args.num_tiles < max_clusters ? args.num_tiles : max_clusters;
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmSFA, tmSFB, tmD, args) != cudaSuccess) return NVFP4_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }

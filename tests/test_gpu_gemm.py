@@ -1,6 +1,8 @@
 """GPU parity of the fused GEMM entry points against the oracle, at sizes the oracle
 finishes in seconds that still span several tiles, several tiles per CTA, and the
-degenerate cases (one tile, one K step, no normalised columns)."""
+degenerate cases (one tile, one K step, no normalised columns). M % 256 == 0 runs the
+CTA-pair kernel, M % 256 == 128 the single-CTA kernel; both appear below, each with more
+tiles than the GPU has SMs (pairs) in at least one case."""
 import numpy as np
 import pytest
 import torch
@@ -22,7 +24,8 @@ def _exact_operands(M, N, K, seed):
     return qa, sa, qb, sb
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 1024), (384, 768, 3072), (2048, 2560, 256)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 1024), (384, 768, 3072), (2048, 2560, 256),
+                                   (1152, 4352, 256), (512, 256, 3072)])
 def test_plain_gemm_is_exact_on_exactly_representable_inputs(M, N, K):
     """E2M1 codes x power-of-two scales: every partial sum is a multiple of 2^-6 below
     2^24 * 2^-6, so FP32 accumulation is exact in any order and the bf16 output must be
@@ -50,7 +53,8 @@ def test_plain_gemm_scales_by_both_global_scales():
     assert np.array_equal(bf16_bits(D), o.bf16_bits(ref))
 
 
-@pytest.mark.parametrize("M,N,K,ldd", [(256, 512, 512, 512), (1280, 768, 768, 800), (2048, 2560, 512, 2560)])
+@pytest.mark.parametrize("M,N,K,ldd", [(256, 512, 512, 512), (1280, 768, 768, 800), (2048, 2560, 512, 2560),
+                                       (384, 512, 512, 512), (1152, 4352, 256, 4352)])
 def test_plain_gemm_matches_oracle(M, N, K, ldd):
     a = wk.activations(M, K, wk.outlier_count(K), seed=1)
     b = wk.weights(N, K, 1 / np.sqrt(K), seed=1)
