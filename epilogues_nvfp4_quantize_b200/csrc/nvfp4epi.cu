@@ -243,14 +243,14 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
     if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     const int64_t units = rows * (cols / 8);
     int64_t blocks = (units + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(info->sm_count) * 8;
+    const int64_t cap = static_cast<int64_t>(info->sm_count) * 4;
     if (blocks > cap) blocks = cap;
     nvfp4::amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(xp, rows, cols, ldx, amax);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     if ((st = launch_status()) != NVFP4_OK) return st;
   }
   const int64_t rows_pad = (rows + 127) / 128 * 128;
-  const int64_t threads = rows_pad * (cols / 8);
+  const int64_t threads = rows_pad * (cols / 64);
   const int64_t blocks = (threads + 255) / 256;
   nvfp4::quantize_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       xp, rows, cols, ldx, (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0, amax, out.gscale,

@@ -1,6 +1,6 @@
 // nvfp4_quantize: bf16 -> NVFP4 (E2M1 codes, E4M3 block scales in the tensor-core scale
-// layout, FP32 per-tensor scale). HBM-bound; one thread owns 8 adjacent values, a lane
-// pair owns one 16-block, and 8 lanes own the 4 blocks of one scale word.
+// layout, FP32 per-tensor scale). HBM-bound: an optional amax pass, then one pass that
+// reads 128 bytes and writes 36 bytes per thread.
 #pragma once
 
 #include "ptx.cuh"
@@ -9,21 +9,34 @@
 namespace nvfp4 {
 
 // amax(|x|) over a rows x cols bf16 tensor, folded into *amax_bits (float bits, the
-// caller zeroes it first) with one atomicMax per block.
+// caller zeroes it first) with one atomicMax per block. Each thread keeps four 16-byte
+// loads in flight per iteration.
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, int64_t ldx,
                                                    unsigned int* __restrict__ amax_bits) {
   const int64_t upr = cols >> 3;  // 16-byte units per row
   const int64_t total = rows * upr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   float m = 0.0f;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = u / upr, c = u - r * upr;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + c * 8));
-    const uint32_t w[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu,
-                           v.w & 0x7FFF7FFFu};
+  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u0 < total; u0 += 4 * stride) {
+    uint4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(bf16_lo(w[i]), bf16_hi(w[i])));
+    for (int i = 0; i < 4; ++i) {
+      const int64_t u = u0 + i * stride;
+      if (u < total) {
+        const int64_t r = u / upr, c = u - r * upr;
+        v[i] = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + c * 8));
+      } else {
+        v[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w[4] = {v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu, v[i].z & 0x7FFF7FFFu,
+                             v[i].w & 0x7FFF7FFFu};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(bf16_lo(w[k]), bf16_hi(w[k])));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -37,9 +50,10 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
   }
 }
 
-// Quantise rows x cols (cols % 64 == 0). Threads cover rows padded to 128 so that the
-// padding scale bytes are written as 0. With `interleave`, output row 2j reads input
-// row j and output row 2j+1 reads input row rows/2 + j.
+// Quantise rows x cols (cols % 64 == 0). One thread owns 64 adjacent values of a row:
+// four 16-blocks, i.e. one 4-byte scale word and 32 bytes of codes. Threads cover rows
+// padded to 128 so that the padding scale words are written as 0. With `interleave`,
+// output row 2j reads input row j and output row 2j+1 reads input row rows/2 + j.
 __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                        int64_t cols, int64_t ldx, int interleave,
                                                        const unsigned int* __restrict__ amax_bits,
@@ -54,46 +68,37 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
     G = *gscale;
   }
   const float enc = scale_encode_factor(G);
-  const int64_t upr = cols >> 3;
+  const int64_t cpr = cols >> 6;  // 64-value groups per row
   const int64_t rows_pad = (rows + 127) & ~static_cast<int64_t>(127);
   const int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (u >= rows_pad * upr) return;  // whole warps only: rows_pad * upr is a multiple of 32
-  const int64_t r = u / upr, c = u - r * upr;
-  const bool valid = r < rows;
-  float v[8];
-  if (valid) {
+  if (u >= rows_pad * cpr) return;
+  const int64_t r = u / cpr, c = u - r * cpr;
+  uint32_t word = 0;
+  if (r < rows) {
     const int64_t src = interleave ? ((r & 1) ? (rows >> 1) + (r >> 1) : (r >> 1)) : r;
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + src * ldx + c * 8));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    const uint4* p = reinterpret_cast<const uint4*>(x + src * ldx + c * 64);
+    uint4 q[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = bf16_lo(w[i]);
-      v[2 * i + 1] = bf16_hi(w[i]);
+    for (int i = 0; i < 8; ++i) q[i] = __ldg(p + i);
+    uint32_t cw[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t w[8] = {q[2 * b].x, q[2 * b].y, q[2 * b].z, q[2 * b].w,
+                             q[2 * b + 1].x, q[2 * b + 1].y, q[2 * b + 1].z, q[2 * b + 1].w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_lo(w[i]);
+        v[2 * i + 1] = bf16_hi(w[i]);
+      }
+      const uint32_t s = quant_block16(v, G, enc, cw[2 * b], cw[2 * b + 1]);
+      word |= s << (8 * b);
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    uint4* dst = reinterpret_cast<uint4*>(codes + r * (cols >> 1) + c * 32);
+    dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
   }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  const uint32_t s = block_scale_code(amax, enc);
-  if (valid) {
-    const uint32_t cw = block_codes8(v, s, G);
-    *reinterpret_cast<uint32_t*>(codes + r * (cols >> 1) + c * 4) = cw;
-  }
-  const int lane = threadIdx.x & 31;
-  const int base = lane & ~7;
-  const uint32_t s0 = __shfl_sync(0xffffffffu, s, base);
-  const uint32_t s1 = __shfl_sync(0xffffffffu, s, base + 2);
-  const uint32_t s2 = __shfl_sync(0xffffffffu, s, base + 4);
-  const uint32_t s3 = __shfl_sync(0xffffffffu, s, base + 6);
-  if ((lane & 7) == 0) {
-    const int64_t kb = c >> 1;  // first 16-block of this 64-column group
-    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(r, kb, cols >> 4)) =
-        s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
-  }
+  *reinterpret_cast<uint32_t*>(sf + sf_word_offset(r, 4 * c, cols >> 4)) = word;
 }
 
 }  // namespace nvfp4
