@@ -18,12 +18,12 @@
 // Epilogues:
 //   PLAIN    y = alpha * acc,  alpha = G_A * G_B
 //   RMSNORM  per head of 128 or 256 columns (sections "Tiles and fragments on Blackwell",
-//            "Why head_dim=256 is hard", "Revisit fusion"): a first touch of TMEM
-//            accumulates the sum of squares of the thread's 128 columns; a 256-wide head
-//            spans the two epilogue warpgroups, which exchange their partial sums through
-//            shared memory (an mbarrier, so the wait stays bounded); a second touch
-//            re-reads TMEM, scales by rstd * w and stores. Columns past n_norm_cols pass
-//            through.
+//            "Why head_dim=256 is hard", "Revisit fusion"): each thread moves its 128
+//            accumulator columns into registers and frees the accumulator; a first pass
+//            over them sums the squares; a 256-wide head spans the two epilogue
+//            warpgroups, which exchange their partial sums through shared memory (an
+//            mbarrier, so the wait stays bounded); a second pass over the same registers
+//            scales by rstd * w and stores. Columns past n_norm_cols pass through.
 //   SWIGLU   accumulator columns come interleaved [g0, u0, g1, u1, ...] from the weight
 //            packing of section "Fusing gated SiLU (SwiGLU)", so each thread computes
 //            silu(g) * u on adjacent columns of its own row; optional NVFP4
@@ -149,8 +149,9 @@ struct EpiCtx {
 };
 
 // Epilogue of one tile: this CTA's 128 rows starting at m0, 256 accumulator columns
-// starting at n0. `release()` is called by every thread once its last TMEM read of the
-// tile has completed (the accumulator may then be overwritten). Returns false if a
+// starting at n0. Each thread first moves its 128 accumulator columns from TMEM into
+// registers (four 32-column loads, one wait) and calls `release()`, so the MMA warp may
+// start the next tile while the op, the rounding and the stores run. Returns false if a
 // bounded wait gave up.
 template <int EPI, class Release>
 __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release release) {
@@ -162,21 +163,23 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
   const int row_in_tile = c.sub * 32 + lane;
   const float alpha = c.alpha;
 
+  uint32_t v[4][32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld32(tcol + 32 * q, v[q]);
+  tmem_ld_wait();
+  release();
+
   if constexpr (EPI == EPI_SWIGLU) {
     uint32_t packed[32];
     uint32_t qc[8];
     uint32_t sfw = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      uint32_t v[32];
-      tmem_ld32(tcol + 32 * q, v);
-      tmem_ld_wait();
-      if (q == 3) release();
       float o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float g = alpha * __uint_as_float(v[2 * j]);
-        const float u = alpha * __uint_as_float(v[2 * j + 1]);
+        const float g = alpha * __uint_as_float(v[q][2 * j]);
+        const float u = alpha * __uint_as_float(v[q][2 * j + 1]);
         o[j] = silu_f32(g) * u;
       }
 #pragma unroll
@@ -212,27 +215,22 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
   } else {
     // PLAIN, or RMSNORM (normalised half) / its passthrough half
     bool norm = false;
-    float rstd = 1.0f;
+    float scale = alpha;  // per-row factor applied to acc: alpha, or alpha * rstd
     if constexpr (EPI == EPI_RMSNORM) {
       norm = col0 < args.n_norm_cols;
       if (norm) {
         float ss = 0.0f;
 #pragma unroll
-        for (int q = 0; q < 4; q += 2) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tcol + 32 * q, v0);
-          tmem_ld32(tcol + 32 * q + 32, v1);
-          tmem_ld_wait();
+        for (int q = 0; q < 4; ++q) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float a = alpha * __uint_as_float(v0[j]);
-            const float b = alpha * __uint_as_float(v1[j]);
+            const float a = alpha * __uint_as_float(v[q][j]);
             ss = fmaf(a, a, ss);
-            ss = fmaf(b, b, ss);
           }
         }
         float mean;
         if (args.head_dim == 256) {
+          // the head's other 128 columns sit in the other warpgroup's registers
           float* slot = c.red + (c.xchg & 1u) * 256;
           slot[c.wg * 128 + row_in_tile] = ss;
           mbar_arrive(c.red_bar);
@@ -244,33 +242,26 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
         } else {
           mean = ss * (1.0f / 128.0f);
         }
-        rstd = rsqrtf(mean + args.eps);
+        scale = alpha * rsqrtf(mean + args.eps);
       }
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tcol + 64 * h, v0);
-      tmem_ld32(tcol + 64 * h + 32, v1);
-      tmem_ld_wait();
-      if (h == 1) release();
       uint32_t p[32];
       if (EPI == EPI_RMSNORM && norm) {
         const float* wp = args.w + col0 + 64 * h;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float2 wa = __ldg(reinterpret_cast<const float2*>(wp + 2 * j));
-          const float2 wb = __ldg(reinterpret_cast<const float2*>(wp + 32 + 2 * j));
-          p[j] = pack_bf16x2(alpha * __uint_as_float(v0[2 * j]) * rstd * wa.x,
-                             alpha * __uint_as_float(v0[2 * j + 1]) * rstd * wa.y);
-          p[16 + j] = pack_bf16x2(alpha * __uint_as_float(v1[2 * j]) * rstd * wb.x,
-                                  alpha * __uint_as_float(v1[2 * j + 1]) * rstd * wb.y);
+        for (int j = 0; j < 32; ++j) {
+          const float2 wv = __ldg(reinterpret_cast<const float2*>(wp + 2 * j));
+          const uint32_t* src = v[2 * h + (j >> 4)];
+          p[j] = pack_bf16x2(__uint_as_float(src[2 * (j & 15)]) * scale * wv.x,
+                             __uint_as_float(src[2 * (j & 15) + 1]) * scale * wv.y);
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          p[j] = pack_bf16x2(alpha * __uint_as_float(v0[2 * j]), alpha * __uint_as_float(v0[2 * j + 1]));
-          p[16 + j] = pack_bf16x2(alpha * __uint_as_float(v1[2 * j]), alpha * __uint_as_float(v1[2 * j + 1]));
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t* src = v[2 * h + (j >> 4)];
+          p[j] = pack_bf16x2(alpha * __uint_as_float(src[2 * (j & 15)]), alpha * __uint_as_float(src[2 * (j & 15) + 1]));
         }
       }
       box_reuse_wait(lane);
