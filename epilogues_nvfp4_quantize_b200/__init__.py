@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     launch_count,
     load,
     nvfp4_quantize,
+    nvfp4_quantize_noalloc,
     quantize_workspace_bytes,
     read_device_status,
     rmsnorm_heads_bf16,

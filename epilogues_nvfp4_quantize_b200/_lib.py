@@ -24,6 +24,7 @@ EXPORTS = (
     "gemm_nvfp4_plain", "gemm_nvfp4_rmsnorm", "gemm_nvfp4_swiglu",
     "rmsnorm_heads_bf16", "swiglu_bf16", "nvfp4_status_string",
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
+    "nvfp4_quantize_noalloc",
 )
 
 
@@ -57,6 +58,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_read_device_status": (i32, [vp]),
         "nvfp4_selftest_bounded_wait": (i32, [i64, vp]),
         "nvfp4_launch_count": (i64, []),
+        "nvfp4_quantize_noalloc": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -168,6 +170,22 @@ def swiglu_bf16(c: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
     py, ldy = _out2d(y)
     _check(load().swiglu_bf16(pc, c.shape[0], c.shape[1] // 2, ldc, py, ldy, _stream(stream)), "swiglu_bf16")
     return y
+
+
+NOALLOC_MAX_VALUES = 268435456
+
+
+def nvfp4_quantize_noalloc(x: torch.Tensor, out: NVFP4Tensor, interleave: bool = False, stream=None) -> NVFP4Tensor:
+    """nvfp4_quantize with the per-tensor scale derived on the device, for callers that
+    cannot allocate device memory: the library keeps the reduction's scratch in its own
+    static device memory, so no workspace is needed (see nvfp4_quantize_noalloc in the
+    header for the size limit and the rule that overlapping calls race)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    _check(load().nvfp4_quantize_noalloc(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0),
+                                         SWIGLU_INTERLEAVE if interleave else 0, out.c(), _stream(stream)),
+           "nvfp4_quantize_noalloc")
+    return out
 
 
 def read_device_status(stream=None) -> int:

@@ -376,3 +376,129 @@ NVFP4_API nvfp4_status nvfp4_selftest_bounded_wait(int64_t limit_ns, cudaStream_
 }
 
 NVFP4_API int64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+// -------------------------------------------------------------------------------------
+// Allocation-free quantiser: nvfp4_quantize with compute_amax = 1, whose scratch (one
+// partial maximum per block of 16384 input values, then the tensor's amax) lives in a
+// file-scope device array instead of a caller workspace.
+// -------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoAllocPartials = 16384;                     // partial maxima the array holds
+constexpr int64_t kNoAllocUnitsPerBlock = 256 * 8;          // 16-byte units per partial (16384 values)
+constexpr int64_t kNoAllocMaxValues = static_cast<int64_t>(kNoAllocPartials) * kNoAllocUnitsPerBlock * 8;
+static_assert(kNoAllocMaxValues == NVFP4_NOALLOC_MAX_VALUES, "limit stated in the header");
+
+// [0, kNoAllocPartials): partial maxima; [kNoAllocPartials]: the tensor's amax (float bits).
+// Every GPU that loads the library holds these 64 KB until the process exits.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartials + 64];
+
+float* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// One partial maximum of |x| per block: block b covers 16-byte units
+// [b * 2048, (b + 1) * 2048) of the row-major rows x cols view. Written, not accumulated.
+__global__ void __launch_bounds__(256) noalloc_amax_partial_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                                   int64_t cols, int64_t ldx,
+                                                                   float* __restrict__ partials) {
+  const int64_t upr = cols >> 3;
+  const int64_t total = rows * upr;
+  const int64_t base = blockIdx.x * kNoAllocUnitsPerBlock;
+  float m = 0.0f;
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t u = base + i * 256 + threadIdx.x;
+    if (u < total) {
+      const int64_t r = u / upr, c = u - r * upr;
+      v[i] = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + c * 8));
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t w[4] = {v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu, v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(nvfp4::bf16_lo(w[k]), nvfp4::bf16_hi(w[k])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int i = 0; i < 8; ++i) b = fmaxf(b, wmax[i]);
+    partials[blockIdx.x] = b;
+  }
+}
+
+// Maximum of the n partials, written as float bits to *amax_bits.
+__global__ void __launch_bounds__(256) noalloc_amax_reduce_kernel(const float* __restrict__ partials, int n,
+                                                                  unsigned int* __restrict__ amax_bits) {
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < n; i += 256) m = fmaxf(m, partials[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int i = 0; i < 8; ++i) b = fmaxf(b, wmax[i]);
+    *amax_bits = __float_as_uint(b);
+  }
+}
+
+// Device address of the scratch array on device `dev` (looked up once per device, with
+// that device current).
+nvfp4_status noalloc_scratch(int dev, float** out) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NVFP4_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ldx, int flags,
+                                              nvfp4_tensor out, cudaStream_t stream) {
+  if (x == nullptr || out.codes == nullptr || out.sf == nullptr || out.gscale == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~NVFP4_SWIGLU_INTERLEAVE) return NVFP4_ERR_INVALID_ARG;
+  if (out.rows != rows || out.cols != cols) return NVFP4_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || cols % 64 != 0 || ldx < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((flags & NVFP4_SWIGLU_INTERLEAVE) && (rows % 2) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  // the scratch array holds one partial maximum per 16384 values
+  if (rows > kNoAllocMaxValues / cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx % 8) != 0 || !aligned16(out.codes) || (reinterpret_cast<uintptr_t>(out.sf) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  float* scratch;
+  if ((st = noalloc_scratch(dev, &scratch)) != NVFP4_OK) return st;
+
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  const int64_t units = rows * (cols / 8);
+  const int blocks = static_cast<int>((units + kNoAllocUnitsPerBlock - 1) / kNoAllocUnitsPerBlock);
+  unsigned int* amax_bits = reinterpret_cast<unsigned int*>(scratch + kNoAllocPartials);
+  noalloc_amax_partial_kernel<<<blocks, 256, 0, stream>>>(xp, rows, cols, ldx, scratch);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if ((st = launch_status()) != NVFP4_OK) return st;
+  noalloc_amax_reduce_kernel<<<1, 256, 0, stream>>>(scratch, blocks, amax_bits);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if ((st = launch_status()) != NVFP4_OK) return st;
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t threads = rows_pad * (cols / 64);
+  nvfp4::quantize_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      xp, rows, cols, ldx, (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0, amax_bits, out.gscale,
+      static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}

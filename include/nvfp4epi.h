@@ -153,6 +153,31 @@ nvfp4_status rmsnorm_heads_bf16(const void* x, int64_t rows, int64_t ldx, const 
 nvfp4_status swiglu_bf16(const void* c, int64_t rows, int64_t nh, int64_t ldc,
                          void* y, int64_t ldy, cudaStream_t stream);
 
+/*
+ * Allocation-free variant of nvfp4_quantize with compute_amax = 1. This entry point has no
+ * counterpart on the page; it exists for callers that cannot allocate device memory: code
+ * embedded in a host application that owns the whole GPU and hands out only its own
+ * buffers (a serving engine that reserves device memory up front), and latency-critical
+ * paths where a cudaMalloc, which may synchronise the device, is not acceptable. The caller
+ * still provides x and `out`; the scratch the amax reduction needs (one partial maximum per
+ * 16384 input values, then the tensor's amax) lives in a 64 KB array of static device
+ * memory inside this library, which every GPU that loads the library holds until exit.
+ * Results are bit for bit those of nvfp4_quantize(..., compute_amax = 1, ...).
+ *   - rows * cols must not exceed NVFP4_NOALLOC_MAX_VALUES, otherwise
+ *     NVFP4_ERR_UNSUPPORTED_SHAPE and nothing is launched; the other rules are those of
+ *     nvfp4_quantize.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array and leave their values in it. Every value a call reads is
+ *     written earlier by the same call, so nothing needs clearing, but calls whose kernels
+ *     overlap on the GPU (different streams, or different host threads) race on the array
+ *     and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ */
+#define NVFP4_NOALLOC_MAX_VALUES 268435456LL /* 16384 partial maxima x 16384 values */
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                    int flags, nvfp4_tensor out, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char* nvfp4_status_string(nvfp4_status status);
 
