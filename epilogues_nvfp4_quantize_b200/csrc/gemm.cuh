@@ -13,7 +13,9 @@
 // Warp roles (320 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
 // and MMA issuer. Epilogue warp w reads TMEM lanes 32*(w%4).. (its 32 output rows) and
 // columns 128*(w/4).. (its half of the 256-column tile); each thread owns one output row.
-// Results go through a 128-byte-swizzled staging box and a TMA store.
+// Results go through a 128-byte-swizzled staging box and a TMA store. Two accumulator
+// buffers in TMEM let the MMAs of tile i+1 run while the epilogue of tile i reads its
+// buffer.
 //
 // Epilogues:
 //   PLAIN    y = alpha * acc,  alpha = G_A * G_B
@@ -51,9 +53,16 @@ constexpr int NUM_THREADS = EPI_THREADS + 64;
 constexpr int BOX_BYTES = 32 * 128;     // one staging box: 32 rows x 128 bytes
 constexpr int RED_BYTES = 2 * 2 * 128 * 4;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;    // 256 fp32 columns
-constexpr uint32_t SFA_COL = 256;  // 4 MMAs x 4 columns
-constexpr uint32_t SFB_COL = 272;  // 4 MMAs x 8 columns
+// Two 256-column FP32 accumulators that overlap in 48 columns, so that both fit beside the
+// 48 columns of block scales: buffer 0 = [0, 256), buffer 1 = [208, 464). The overlap
+// [208, 256) is held by warpgroup 1 of buffer 0 and warpgroup 0 of buffer 1; the next
+// tile may start once that warpgroup has read its columns.
+constexpr uint32_t ACC_COL1 = 208;
+constexpr uint32_t SFA_COL = 464;  // 4 MMAs x 4 columns
+constexpr uint32_t SFB_COL = 480;  // 4 MMAs x 8 columns
+__host__ __device__ constexpr uint32_t acc_col(uint32_t buf) { return buf ? ACC_COL1 : 0u; }
+__host__ __device__ constexpr int overlap_wg(uint32_t buf) { return buf ? 0 : 1; }
+static_assert(ACC_COL1 + 256 <= SFA_COL && SFB_COL + 32 <= TMEM_COLS, "TMEM plan");
 }  // namespace gemm_cfg
 
 // Shared-memory plan of a kernel with S stages of B_ROWS rows of B per CTA.
@@ -67,7 +76,7 @@ struct SmemPlan {
   static constexpr int OFF_EPI = S * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
   static constexpr int OFF_BAR = OFF_RED + gemm_cfg::RED_BYTES;
-  static constexpr int NUM_BARS = 2 * S + 4;
+  static constexpr int NUM_BARS = 2 * S + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -75,6 +84,30 @@ struct SmemPlan {
 };
 using PlanSingle = SmemPlan<3, 256>;
 using PlanPair = SmemPlan<5, 128>;
+
+// Accumulator hand-off between the MMA warp and the epilogue: per buffer one "full"
+// barrier (MMA commit) and one "empty" barrier per warpgroup (one arrival per warp of that
+// warpgroup, in each CTA of the pair).
+struct AccBars {
+  uint64_t* full;   // [2]
+  uint64_t* empty;  // [2][2]: empty[2 * buf + wg]
+  __device__ __forceinline__ uint64_t* emp(uint32_t buf, int wg) const { return empty + 2 * buf + wg; }
+};
+
+// MMA side: before tile j (buffer j & 1) may overwrite its accumulator, both warpgroups
+// must have read the buffer's previous tile (j - 2), and the warpgroup holding the
+// overlap must have read tile j - 1 (the other buffer).
+__device__ __forceinline__ bool acc_acquire(const AccBars& a, uint32_t j, volatile int* abort_flag,
+                                            uint64_t limit, int where) {
+  const uint32_t b = j & 1u, u = j >> 1;
+  if (!mbar_wait(a.emp(b, 0), (u & 1u) ^ 1u, abort_flag, limit, where)) return false;
+  if (!mbar_wait(a.emp(b, 1), (u & 1u) ^ 1u, abort_flag, limit, where)) return false;
+  if (j >= 1) {
+    const uint32_t bp = b ^ 1u, up = (j - 1) >> 1;
+    if (!mbar_wait(a.emp(bp, gemm_cfg::overlap_wg(bp)), up & 1u, abort_flag, limit, where)) return false;
+  }
+  return true;
+}
 
 struct GemmArgs {
   const uint8_t* sfa;
@@ -154,11 +187,11 @@ struct EpiCtx {
 // start the next tile while the op, the rounding and the stores run. Returns false if a
 // bounded wait gave up.
 template <int EPI, class Release>
-__device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release release) {
+__device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, int n0, Release release) {
   using namespace gemm_cfg;
   const GemmArgs& args = *c.args;
   const int lane = c.lane;
-  const uint32_t tcol = c.t_row + ACC_COL + c.wg * 128;
+  const uint32_t tcol = c.t_row + acc_col(buf) + c.wg * 128;
   const int col0 = n0 + c.wg * 128;
   const int row_in_tile = c.sub * 32 + lane;
   const float alpha = c.alpha;
@@ -312,10 +345,9 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* red_bar = acc_full + 2;
-  uint64_t* drain_bar = acc_full + 3;
+  AccBars acc{empty + STAGES, empty + STAGES + 2};
+  uint64_t* red_bar = empty + STAGES + 6;
+  uint64_t* drain_bar = empty + STAGES + 7;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
@@ -328,8 +360,11 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, EPI_WARPS);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc.full[b], 1);
+      mbar_init(acc.emp(b, 0), EPI_WARPS / 2);
+      mbar_init(acc.emp(b, 1), EPI_WARPS / 2);
+    }
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -411,14 +446,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_nvfp4(BM, BN);
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0, j = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, limit, 2)) {
+      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++j) {
+        if (!acc_acquire(acc, j, abort_flag, limit, 2)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t d_tmem = tmem + acc_col(j & 1u);
         for (int kt = 0; kt < ktiles; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3)) {
             ok = false;
@@ -440,7 +476,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
 #pragma unroll
           for (int kb = 0; kb < BK / 64; ++kb) {
             // +32 bytes along K per 64 FP4 values: +2 in the descriptor's address field
-            tc_mma_nvfp4(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
+            tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
                          tmem + SFB_COL + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
@@ -450,8 +486,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           }
         }
         if (!ok) break;
-        tc_commit(acc_full);
-        acc_phase ^= 1u;
+        tc_commit(&acc.full[j & 1u]);
       }
       if (!ok) {
         tc_commit(drain_bar);
@@ -461,20 +496,20 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue
     EpiCtx c = make_epi_ctx(args, &tmD, tmem, smem, P::OFF_EPI, P::OFF_RED, red_bar, abort_flag);
-    auto release = [&]() {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-    };
-    uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
+    uint32_t j = 0;
+    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, ++j) {
       int tm, tn;
       tile_coords(args, t, tm, tn);
+      const uint32_t b = j & 1u;
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc.emp(b, c.wg));
+      };
       // every lane waits; the warp leaves together if any lane gave up
-      if (!__all_sync(0xffffffffu, mbar_wait(acc_full, acc_phase, abort_flag, limit, 4))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc.full[b], (j >> 1) & 1u, abort_flag, limit, 4))) break;
       tc_fence_after();
-      if (!epilogue_tile<EPI>(c, tm * BM, tn * BN, release)) break;
-      acc_phase ^= 1u;
+      if (!epilogue_tile<EPI>(c, b, tm * BM, tn * BN, release)) break;
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -504,10 +539,9 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* red_bar = acc_full + 2;
-  uint64_t* drain_bar = acc_full + 3;
+  AccBars acc{empty + STAGES, empty + STAGES + 2};  // leader's empty barriers count both CTAs
+  uint64_t* red_bar = empty + STAGES + 6;
+  uint64_t* drain_bar = empty + STAGES + 7;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
@@ -524,8 +558,11 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
       mbar_init(&full[s], 1);   // leader's: one expect-tx arrival, both CTAs' bytes
       mbar_init(&empty[s], 1);  // one multicast commit per use
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * EPI_WARPS);  // leader's: one arrival per epilogue warp of the pair
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc.full[b], 1);
+      mbar_init(acc.emp(b, 0), EPI_WARPS);  // leader's: one arrival per warp of the warpgroup, per CTA
+      mbar_init(acc.emp(b, 1), EPI_WARPS);
+    }
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -612,14 +649,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     if (leader && lane == 0) {
       const uint32_t idesc = idesc_nvfp4(2 * BM, BN);
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0, j = 0;
       bool ok = true;
-      for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, limit, 22)) {
+      for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters, ++j) {
+        if (!acc_acquire(acc, j, abort_flag, limit, 22)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t d_tmem = tmem + acc_col(j & 1u);
         for (int kt = 0; kt < ktiles; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25)) {
             ok = false;
@@ -641,7 +679,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           const uint64_t bdesc = smem_desc_sw128(b_addr);
 #pragma unroll
           for (int kb = 0; kb < BK / 64; ++kb) {
-            tc_mma_nvfp4_pair(tmem + ACC_COL, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
+            tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
                               tmem + SFB_COL + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
@@ -651,8 +689,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           }
         }
         if (!ok) break;
-        tc_commit_pair(acc_full, 0x3);
-        acc_phase ^= 1u;
+        tc_commit_pair(&acc.full[j & 1u], 0x3);
       }
       if (!ok) {
         tc_commit_pair(drain_bar, 0x1);
@@ -662,20 +699,20 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     EpiCtx c = make_epi_ctx(args, &tmD, tmem, smem, P::OFF_EPI, P::OFF_RED, red_bar, abort_flag);
-    const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
-    auto release = [&]() {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
-    };
-    uint32_t acc_phase = 0;
-    for (int t = cluster_id; t < args.num_tiles; t += num_clusters) {
+    uint32_t j = 0;
+    for (int t = cluster_id; t < args.num_tiles; t += num_clusters, ++j) {
       int tm, tn;
       tile_coords(args, t, tm, tn);
-      if (!__all_sync(0xffffffffu, mbar_wait(acc_full, acc_phase, abort_flag, limit, 27))) break;
+      const uint32_t b = j & 1u;
+      const uint32_t leader_empty = mapa_shared(smem_u32(acc.emp(b, c.wg)), 0);
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_empty);
+      };
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc.full[b], (j >> 1) & 1u, abort_flag, limit, 27))) break;
       tc_fence_after();
-      if (!epilogue_tile<EPI>(c, tm * 256 + 128 * static_cast<int>(rank), tn * BN, release)) break;
-      acc_phase ^= 1u;
+      if (!epilogue_tile<EPI>(c, b, tm * 256 + 128 * static_cast<int>(rank), tn * BN, release)) break;
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
