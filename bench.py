@@ -49,6 +49,24 @@ def workload_desc(M: int) -> str:
             f"SwiGLU + NVFP4 re-quantisation -> FFN-down GEMM K={K_DOWN} N={K_IN}")
 
 
+# DRAM bytes (read + write) per launch of the FFN-up fused GEMM at M=16384, from the ncu
+# capture summarised in profiles/, keyed by a hash of the GEMM's device sources: a value
+# taken on another version of the kernel is not reported.
+TRAFFIC_BY_SOURCE = {
+    "49979b758997f807": 146.3e6,
+}
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "epilogues_nvfp4_quantize_b200", "csrc")
+    for f in ("gemm.cuh", "ptx.cuh", "codec.cuh", "unfused.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -76,7 +94,7 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
-                                          "-lms", "200", "-i", str(self.gpu)], stdout=self.fh,
+                                          "-lms", "50", "-i", str(self.gpu)], stdout=self.fh,
                                          stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except (OSError, FileNotFoundError):
@@ -303,9 +321,13 @@ def run_cuda(args):
                    "K_down": K_DOWN, "head_dim": HD, "global_batch_tokens": M * world,
                    "parallelism": f"dp{world} (independent token batches, no collective)",
                    "l2": "no flush: per-step inputs (x 100.7 MB + packed weights 75 MB) exceed the 126 MB L2"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel<SWIGLU> (FFN-up, requant)",
+        "roofline": {"bound": "tensor",
+                     "kernel": ("gemm_nvfp4_pair_kernel<EPI_SWIGLU>" if M % 256 == 0 else
+                                "gemm_nvfp4_kernel<EPI_SWIGLU>") + " (FFN-up, SwiGLU + NVFP4 re-quantisation)",
                      "achieved": round(up_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(up_tflops / fp4_peak, 4), "traffic": args.traffic,
+                     "frac": round(up_tflops / fp4_peak, 4),
+                     "traffic": args.traffic if args.traffic is not None else
+                     (TRAFFIC_BY_SOURCE.get(gemm_source_hash()) if M == 16384 else None),
                      "peak_source": f"{pk['source']} bf16 {pk['bf16']} TFLOP/s x {FP4_PER_BF16} (nominal dense "
                                     f"FP4:BF16 ratio), burst figure"},
         "kernels": kernels,
@@ -347,7 +369,7 @@ def run_cuda(args):
             out_host.copy_(layer.out, non_blocking=True)
 
         barrier()
-        t_e2e = time_loop(e2e_step, max(2, K // 2), 2, torch)
+        t_e2e = time_loop(e2e_step, max(2, min(K // 2, 100)), 3, torch)
         te = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
@@ -462,7 +484,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=600)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--M", type=int, default=16384, help="tokens per GPU per step")
