@@ -53,7 +53,6 @@ def workload_desc(M: int) -> str:
 # capture summarised in profiles/, keyed by a hash of the GEMM's device sources: a value
 # taken on another version of the kernel is not reported.
 TRAFFIC_BY_SOURCE = {
-    "49979b758997f807": 146.3e6,
 }
 
 

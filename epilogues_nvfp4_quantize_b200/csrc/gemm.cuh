@@ -10,9 +10,14 @@
 //       stages its own 128 rows of A and 128 of the 256 rows of B, so a CTA moves
 //       38 KB per K step of 256 for 128 x 256 x 256 MMA work (5-stage ring);
 //   gemm_nvfp4_kernel       (M % 256 == 128) one CTA per 128 x 256 tile (3-stage ring).
-// Warp roles (320 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
-// and MMA issuer. Epilogue warp w reads TMEM lanes 32*(w%4).. (its 32 output rows) and
-// columns 128*(w/4).. (its half of the 256-column tile); each thread owns one output row.
+// Warp roles (384 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
+// and MMA issuer, warps 10-11 copy the block scales from shared memory into TMEM
+// (tcgen05.cp). Each tcgen05 instruction holds up the warp that issues it for a while;
+// issued from their own warps (on other SM sub-partitions) the 12 scale copies of a K step
+// overlap the 4 MMAs instead of queueing in front of them. Two TMEM scale slots let the
+// copies of K step g+1 run while the MMAs of step g read the other slot.
+// Epilogue warp w reads TMEM lanes 32*(w%4).. (its 32 output rows) and columns
+// 128*(w/4).. (its half of the 256-column tile); each thread owns one output row.
 // Results go through a 128-byte-swizzled staging box and a TMA store. Two accumulator
 // buffers in TMEM let the MMAs of tile i+1 run while the epilogue of tile i reads its
 // buffer.
@@ -49,20 +54,26 @@ constexpr int BK_BYTES = BK / 2;        // 128: one swizzle row
 constexpr int SF_UNIT = 512;            // scales of 128 rows x 64 K
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int NUM_THREADS = EPI_THREADS + 64;
+constexpr int COPY_WARPS = 2;
+constexpr int NUM_THREADS = EPI_THREADS + 64 + 32 * COPY_WARPS;
+constexpr int PRODUCER_WARP = EPI_WARPS;
+constexpr int MMA_WARP = EPI_WARPS + 1;
+constexpr int COPY_WARP0 = EPI_WARPS + 2;
 constexpr int BOX_BYTES = 32 * 128;     // one staging box: 32 rows x 128 bytes
 constexpr int RED_BYTES = 2 * 2 * 128 * 4;
 constexpr uint32_t TMEM_COLS = 512;
-// Two 256-column FP32 accumulators that overlap in 48 columns, so that both fit beside the
-// 48 columns of block scales: buffer 0 = [0, 256), buffer 1 = [208, 464). The overlap
-// [208, 256) is held by warpgroup 1 of buffer 0 and warpgroup 0 of buffer 1; the next
-// tile may start once that warpgroup has read its columns.
-constexpr uint32_t ACC_COL1 = 208;
-constexpr uint32_t SFA_COL = 464;  // 4 MMAs x 4 columns
-constexpr uint32_t SFB_COL = 480;  // 4 MMAs x 8 columns
+// Two 256-column FP32 accumulators that overlap in 96 columns, so that both fit beside two
+// 48-column slots of block scales: buffer 0 = [0, 256), buffer 1 = [160, 416), scale slots
+// at 416 and 464. The overlap [160, 256) is held by warpgroup 1 of buffer 0 and warpgroup 0
+// of buffer 1; the next tile may start once that warpgroup has read its columns.
+constexpr uint32_t ACC_COL1 = 160;
+constexpr uint32_t SF_SLOT0 = 416;
+constexpr uint32_t SF_SLOT_COLS = 48;  // per K step: SFA 4 MMAs x 4 columns, then SFB 4 MMAs x 8
+constexpr uint32_t SFB_OFF = 16;
 __host__ __device__ constexpr uint32_t acc_col(uint32_t buf) { return buf ? ACC_COL1 : 0u; }
 __host__ __device__ constexpr int overlap_wg(uint32_t buf) { return buf ? 0 : 1; }
-static_assert(ACC_COL1 + 256 <= SFA_COL && SFB_COL + 32 <= TMEM_COLS, "TMEM plan");
+__host__ __device__ constexpr uint32_t sf_slot(uint32_t s) { return SF_SLOT0 + SF_SLOT_COLS * s; }
+static_assert(ACC_COL1 + 256 <= SF_SLOT0 && ACC_COL1 >= 128 && sf_slot(2) <= TMEM_COLS, "TMEM plan");
 }  // namespace gemm_cfg
 
 // Shared-memory plan of a kernel with S stages of B_ROWS rows of B per CTA.
@@ -76,7 +87,7 @@ struct SmemPlan {
   static constexpr int OFF_EPI = S * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
   static constexpr int OFF_BAR = OFF_RED + gemm_cfg::RED_BYTES;
-  static constexpr int NUM_BARS = 2 * S + 8;
+  static constexpr int NUM_BARS = 2 * S + 14;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -84,6 +95,18 @@ struct SmemPlan {
 };
 using PlanSingle = SmemPlan<3, 256>;
 using PlanPair = SmemPlan<5, 128>;
+
+// Barriers past the stage ring (full[S], empty[S]), at empty + S + index.
+namespace bar_idx {
+constexpr int ACC_FULL = 0;   // [2]
+constexpr int ACC_EMPTY = 2;  // [2][2]
+constexpr int RED = 6;
+constexpr int DRAIN = 7;      // MMA warp's own drain on give-up
+constexpr int SF_FULL = 8;    // [2] scale slot filled (one commit per copy warp)
+constexpr int SF_EMPTY = 10;  // [2] scale slot read by the MMAs (one MMA commit)
+constexpr int CP_DRAIN = 12;  // [COPY_WARPS] copy warps' own drain on give-up
+}  // namespace bar_idx
+static_assert(bar_idx::CP_DRAIN + gemm_cfg::COPY_WARPS <= 14, "barrier plan");
 
 // Accumulator hand-off between the MMA warp and the epilogue: per buffer one "full"
 // barrier (MMA commit) and one "empty" barrier per warpgroup (one arrival per warp of that
@@ -107,6 +130,80 @@ __device__ __forceinline__ bool acc_acquire(const AccBars& a, uint32_t j, volati
     if (!mbar_wait(a.emp(bp, gemm_cfg::overlap_wg(bp)), up & 1u, abort_flag, limit, where)) return false;
   }
   return true;
+}
+
+// K steps run by a CTA (or CTA pair) that takes tiles first, first + stride, ...
+__device__ __forceinline__ uint32_t ksteps_of(int num_tiles, int K, int first, int stride) {
+  const int tiles = first < num_tiles ? (num_tiles - 1 - first) / stride + 1 : 0;
+  return static_cast<uint32_t>(tiles) * static_cast<uint32_t>(K / gemm_cfg::BK);
+}
+
+// Scale-copy warp `cw` (one elected lane). For K step g in stage `stage`: once the stage's
+// data has landed and the MMAs of step g - 2 have finished reading scale slot g % 2, copy its
+// share of the step's 12 scale units (unit i goes to warp i % COPY_WARPS) into that slot and
+// commit to sf_full[g % 2]. Slot layout: SFA of MMA q at columns 4q, SFB rows 0-127 of MMA q
+// at 16 + 8q, rows 128-255 at 16 + 8q + 4. In a CTA pair the leader copies for both CTAs and
+// the commits go to the leader's barriers only. Returns false if a bounded wait gave up
+// (after waiting, bounded, for its own copies).
+template <bool PAIR, int STAGES, int STAGE_BYTES, int SF_OFF, int SFB_HALF>
+__device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* full, uint64_t* bars, uint32_t tmem,
+                                                int cw, uint32_t nsteps, volatile int* abort_flag, uint64_t limit,
+                                                int where) {
+  using namespace gemm_cfg;
+  uint64_t* sf_full = bars + bar_idx::SF_FULL;
+  uint64_t* sf_empty = bars + bar_idx::SF_EMPTY;
+  int stage = 0;
+  uint32_t phase = 0;
+  bool ok = true;
+  for (uint32_t g = 0; g < nsteps; ++g) {
+    const uint32_t s = g & 1u, u = g >> 1;
+    if (!mbar_wait(&full[stage], phase, abort_flag, limit, where) ||
+        !mbar_wait(&sf_empty[s], (u & 1u) ^ 1u, abort_flag, limit, where + 1)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    const uint32_t sfa = smem_u32(smem + stage * STAGE_BYTES) + SF_OFF;
+    const uint32_t sfb = sfa + (BK / 64) * SF_UNIT;
+    const uint32_t slot = tmem + sf_slot(s);
+#pragma unroll
+    for (int i = 0; i < 3 * (BK / 64); ++i) {
+      if (i % COPY_WARPS != cw) continue;
+      const int q = i / 3, r = i % 3;
+      const uint32_t dst = r == 0 ? slot + 4 * q : slot + SFB_OFF + 8 * q + 4 * (r - 1);
+      const uint32_t src = r == 0 ? sfa + q * SF_UNIT : sfb + (r - 1) * SFB_HALF + q * SF_UNIT;
+      if constexpr (PAIR) {
+        tc_copy_scales_pair(dst, smem_desc_scales(src));
+      } else {
+        tc_copy_scales(dst, smem_desc_scales(src));
+      }
+    }
+    if constexpr (PAIR) {
+      tc_commit_pair(&sf_full[s], 0x1);
+    } else {
+      tc_commit(&sf_full[s]);
+    }
+    if (++stage == STAGES) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+  if (ok) {
+    // Tail: wait for the MMA commits that release the last two slots, so that no arrival
+    // reaches this CTA's barriers after it exits.
+    for (uint32_t g = nsteps; g < nsteps + 2; ++g) {
+      if (!mbar_wait(&sf_empty[g & 1u], ((g >> 1) & 1u) ^ 1u, abort_flag, limit, where + 1)) break;
+    }
+  } else {
+    uint64_t* drain = bars + bar_idx::CP_DRAIN + cw;
+    if constexpr (PAIR) {
+      tc_commit_pair(drain, 0x1);
+    } else {
+      tc_commit(drain);
+    }
+    (void)mbar_wait(drain, 0, nullptr, limit, where + 2);
+  }
+  return ok;
 }
 
 struct GemmArgs {
@@ -348,6 +445,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   AccBars acc{empty + STAGES, empty + STAGES + 2};
   uint64_t* red_bar = empty + STAGES + 6;
   uint64_t* drain_bar = empty + STAGES + 7;
+  uint64_t* xbars = empty + STAGES;  // bar_idx layout
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
@@ -367,6 +465,11 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     }
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&xbars[bar_idx::SF_FULL + b], COPY_WARPS);
+      mbar_init(&xbars[bar_idx::SF_EMPTY + b], 1);
+    }
+    for (int w = 0; w < COPY_WARPS; ++w) mbar_init(&xbars[bar_idx::CP_DRAIN + w], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -446,7 +549,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_nvfp4(BM, BN);
       int stage = 0;
-      uint32_t phase = 0, j = 0;
+      uint32_t phase = 0, j = 0, g = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++j) {
         if (!acc_acquire(acc, j, abort_flag, limit, 2)) {
@@ -455,31 +558,27 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc_col(j & 1u);
-        for (int kt = 0; kt < ktiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3)) {
+        for (int kt = 0; kt < ktiles; ++kt, ++g) {
+          const uint32_t sl = g & 1u;
+          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3) ||
+              !mbar_wait(&xbars[bar_idx::SF_FULL + sl], (g >> 1) & 1u, abort_flag, limit, 5)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
           const uint32_t b_addr = a_addr + P::A_BYTES;
-          const uint32_t sfa_addr = b_addr + P::B_BYTES;
-          const uint32_t sfb_addr = sfa_addr + P::SFA_BYTES;
-#pragma unroll
-          for (int j = 0; j < BK / 64; ++j) {
-            tc_copy_scales(tmem + SFA_COL + 4 * j, smem_desc_scales(sfa_addr + j * SF_UNIT));
-            tc_copy_scales(tmem + SFB_COL + 8 * j, smem_desc_scales(sfb_addr + j * SF_UNIT));
-            tc_copy_scales(tmem + SFB_COL + 8 * j + 4, smem_desc_scales(sfb_addr + P::SFB_BYTES / 2 + j * SF_UNIT));
-          }
+          const uint32_t slot = tmem + sf_slot(sl);
           const uint64_t adesc = smem_desc_sw128(a_addr);
           const uint64_t bdesc = smem_desc_sw128(b_addr);
 #pragma unroll
           for (int kb = 0; kb < BK / 64; ++kb) {
             // +32 bytes along K per 64 FP4 values: +2 in the descriptor's address field
-            tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
-                         tmem + SFB_COL + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
+            tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, slot + 4 * kb, slot + SFB_OFF + 8 * kb,
+                         (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
+          tc_commit(&xbars[bar_idx::SF_EMPTY + sl]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -492,6 +591,13 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
         tc_commit(drain_bar);
         (void)mbar_wait(drain_bar, 0, nullptr, limit, 12);
       }
+    }
+  } else if (warp >= COPY_WARP0) {
+    // ------------------------------------------------------------------ scale copies
+    if (lane == 0) {
+      (void)scale_copy_loop<false, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
+          abort_flag, limit, 14);
     }
   } else {
     // ------------------------------------------------------------------ epilogue
@@ -542,6 +648,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   AccBars acc{empty + STAGES, empty + STAGES + 2};  // leader's empty barriers count both CTAs
   uint64_t* red_bar = empty + STAGES + 6;
   uint64_t* drain_bar = empty + STAGES + 7;
+  uint64_t* xbars = empty + STAGES;  // bar_idx layout
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
@@ -565,6 +672,11 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     }
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&xbars[bar_idx::SF_FULL + b], COPY_WARPS);  // leader's: the leader's copy warps
+      mbar_init(&xbars[bar_idx::SF_EMPTY + b], 1);
+    }
+    for (int w = 0; w < COPY_WARPS; ++w) mbar_init(&xbars[bar_idx::CP_DRAIN + w], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -649,7 +761,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     if (leader && lane == 0) {
       const uint32_t idesc = idesc_nvfp4(2 * BM, BN);
       int stage = 0;
-      uint32_t phase = 0, j = 0;
+      uint32_t phase = 0, j = 0, g = 0;
       bool ok = true;
       for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters, ++j) {
         if (!acc_acquire(acc, j, abort_flag, limit, 22)) {
@@ -658,31 +770,26 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc_col(j & 1u);
-        for (int kt = 0; kt < ktiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25)) {
+        for (int kt = 0; kt < ktiles; ++kt, ++g) {
+          const uint32_t sl = g & 1u;
+          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25) ||
+              !mbar_wait(&xbars[bar_idx::SF_FULL + sl], (g >> 1) & 1u, abort_flag, limit, 28)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
           const uint32_t b_addr = a_addr + P::A_BYTES;
-          const uint32_t sfa_addr = b_addr + P::B_BYTES;
-          const uint32_t sfb_addr = sfa_addr + P::SFA_BYTES;
-#pragma unroll
-          for (int j = 0; j < BK / 64; ++j) {
-            tc_copy_scales_pair(tmem + SFA_COL + 4 * j, smem_desc_scales(sfa_addr + j * SF_UNIT));
-            tc_copy_scales_pair(tmem + SFB_COL + 8 * j, smem_desc_scales(sfb_addr + j * SF_UNIT));
-            tc_copy_scales_pair(tmem + SFB_COL + 8 * j + 4,
-                                smem_desc_scales(sfb_addr + P::SFB_BYTES / 2 + j * SF_UNIT));
-          }
+          const uint32_t slot = tmem + sf_slot(sl);
           const uint64_t adesc = smem_desc_sw128(a_addr);
           const uint64_t bdesc = smem_desc_sw128(b_addr);
 #pragma unroll
           for (int kb = 0; kb < BK / 64; ++kb) {
-            tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + SFA_COL + 4 * kb,
-                              tmem + SFB_COL + 8 * kb, (kt > 0 || kb > 0) ? 1u : 0u);
+            tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, slot + 4 * kb, slot + SFB_OFF + 8 * kb,
+                              (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
+          tc_commit_pair(&xbars[bar_idx::SF_EMPTY + sl], 0x1);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -695,6 +802,13 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
         tc_commit_pair(drain_bar, 0x1);
         (void)mbar_wait(drain_bar, 0, nullptr, limit, 26);
       }
+    }
+  } else if (warp >= COPY_WARP0) {
+    // ------------------------------------------------------------------ scale copies (leader only)
+    if (leader && lane == 0) {
+      (void)scale_copy_loop<true, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
+          abort_flag, limit, 31);
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
