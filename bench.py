@@ -328,7 +328,8 @@ def run_cuda(args):
                      "traffic": args.traffic if args.traffic is not None else
                      (TRAFFIC_BY_SOURCE.get(gemm_source_hash()) if M == 16384 else None),
                      "peak_source": f"{pk['source']} bf16 {pk['bf16']} TFLOP/s x {FP4_PER_BF16} (nominal dense "
-                                    f"FP4:BF16 ratio), burst figure"},
+                                    f"FP4:BF16 ratio), burst figure",
+                     "frac_of_sustained": round(up_tflops / (pk["bf16_sustained"] * FP4_PER_BF16), 4)},
         "kernels": kernels,
         "gpu_launches": launches,
         "clocks": clocks,
