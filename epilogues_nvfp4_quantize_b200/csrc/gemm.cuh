@@ -87,7 +87,7 @@ struct SmemPlan {
   static constexpr int OFF_EPI = S * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
   static constexpr int OFF_BAR = OFF_RED + gemm_cfg::RED_BYTES;
-  static constexpr int NUM_BARS = 2 * S + 14;
+  static constexpr int NUM_BARS = 3 * S + 14;  // full, empty, 14 more (bar_idx), scales loaded
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -105,6 +105,7 @@ constexpr int DRAIN = 7;      // MMA warp's own drain on give-up
 constexpr int SF_FULL = 8;    // [2] scale slot filled (one commit per copy warp)
 constexpr int SF_EMPTY = 10;  // [2] scale slot read by the MMAs (one MMA commit)
 constexpr int CP_DRAIN = 12;  // [COPY_WARPS] copy warps' own drain on give-up
+constexpr int SF_LOADED = 14; // [S] a stage's scale units have landed (their own tx count)
 }  // namespace bar_idx
 static_assert(bar_idx::CP_DRAIN + gemm_cfg::COPY_WARPS <= 14, "barrier plan");
 
@@ -139,25 +140,27 @@ __device__ __forceinline__ uint32_t ksteps_of(int num_tiles, int K, int first, i
 }
 
 // Scale-copy warp `cw` (one elected lane). For K step g in stage `stage`: once the stage's
-// data has landed and the MMAs of step g - 2 have finished reading scale slot g % 2, copy its
+// scale units have landed (they have their own barrier, so the copies overlap the arrival
+// of the larger code tiles) and the MMAs of step g - 2 have finished reading scale slot g % 2, copy its
 // share of the step's 12 scale units (unit i goes to warp i % COPY_WARPS) into that slot and
 // commit to sf_full[g % 2]. Slot layout: SFA of MMA q at columns 4q, SFB rows 0-127 of MMA q
 // at 16 + 8q, rows 128-255 at 16 + 8q + 4. In a CTA pair the leader copies for both CTAs and
 // the commits go to the leader's barriers only. Returns false if a bounded wait gave up
 // (after waiting, bounded, for its own copies).
 template <bool PAIR, int STAGES, int STAGE_BYTES, int SF_OFF, int SFB_HALF>
-__device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* full, uint64_t* bars, uint32_t tmem,
+__device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* bars, uint32_t tmem,
                                                 int cw, uint32_t nsteps, volatile int* abort_flag, uint64_t limit,
                                                 int where) {
   using namespace gemm_cfg;
   uint64_t* sf_full = bars + bar_idx::SF_FULL;
   uint64_t* sf_empty = bars + bar_idx::SF_EMPTY;
+  uint64_t* sf_loaded = bars + bar_idx::SF_LOADED;
   int stage = 0;
   uint32_t phase = 0;
   bool ok = true;
   for (uint32_t g = 0; g < nsteps; ++g) {
     const uint32_t s = g & 1u, u = g >> 1;
-    if (!mbar_wait(&full[stage], phase, abort_flag, limit, where) ||
+    if (!mbar_wait(&sf_loaded[stage], phase, abort_flag, limit, where) ||
         !mbar_wait(&sf_empty[s], (u & 1u) ^ 1u, abort_flag, limit, where + 1)) {
       ok = false;
       break;
@@ -300,6 +303,9 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, i
   release();
 
   if constexpr (EPI == EPI_SWIGLU) {
+    // silu(alpha a) * (alpha b) = (a b) alpha^2 / (1 + 2^(-alpha log2(e) a))
+    const float k_exp = -alpha * 1.4426950408889634f;
+    const float alpha2 = alpha * alpha;
     uint32_t packed[32];
     uint32_t qc[8];
     uint32_t sfw = 0;
@@ -308,21 +314,15 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, i
       float o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float g = alpha * __uint_as_float(v[q][2 * j]);
-        const float u = alpha * __uint_as_float(v[q][2 * j + 1]);
-        o[j] = silu_f32(g) * u;
+        const float a = __uint_as_float(v[q][2 * j]);
+        const float b = __uint_as_float(v[q][2 * j + 1]);
+        o[j] = __fdividef(a * b, 1.0f + ex2_approx(a * k_exp)) * alpha2;
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) packed[8 * q + j] = pack_bf16x2(o[2 * j], o[2 * j + 1]);
       if (args.q_codes != nullptr) {
-        float ob[16];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          ob[2 * j] = bf16_lo(packed[8 * q + j]);
-          ob[2 * j + 1] = bf16_hi(packed[8 * q + j]);
-        }
         uint32_t lo, hi;
-        const uint32_t s = quant_block16(ob, c.qG, c.qenc, lo, hi);
+        const uint32_t s = quant_block16_bf16(&packed[8 * q], c.qG, c.qenc, lo, hi);
         qc[2 * q] = lo;
         qc[2 * q + 1] = hi;
         sfw |= s << (8 * q);
@@ -349,12 +349,13 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, i
     if constexpr (EPI == EPI_RMSNORM) {
       norm = col0 < args.n_norm_cols;
       if (norm) {
+        // sum of squares of the raw accumulator; alpha^2 is applied to the mean
         float ss = 0.0f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float a = alpha * __uint_as_float(v[q][j]);
+            const float a = __uint_as_float(v[q][j]);
             ss = fmaf(a, a, ss);
           }
         }
@@ -368,9 +369,9 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, i
             return false;
           ss = slot[row_in_tile] + slot[128 + row_in_tile];
           ++c.xchg;
-          mean = ss * (1.0f / 256.0f);
+          mean = ss * (alpha * alpha * (1.0f / 256.0f));
         } else {
-          mean = ss * (1.0f / 128.0f);
+          mean = ss * (alpha * alpha * (1.0f / 128.0f));
         }
         scale = alpha * rsqrtf(mean + args.eps);
       }
@@ -379,13 +380,15 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, i
     for (int h = 0; h < 2; ++h) {
       uint32_t p[32];
       if (EPI == EPI_RMSNORM && norm) {
-        const float* wp = args.w + col0 + 64 * h;
+        const float4* wp = reinterpret_cast<const float4*>(args.w + col0 + 64 * h);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float2 wv = __ldg(reinterpret_cast<const float2*>(wp + 2 * j));
-          const uint32_t* src = v[2 * h + (j >> 4)];
-          p[j] = pack_bf16x2(__uint_as_float(src[2 * (j & 15)]) * scale * wv.x,
-                             __uint_as_float(src[2 * (j & 15) + 1]) * scale * wv.y);
+        for (int j = 0; j < 16; ++j) {
+          const float4 wv = __ldg(wp + j);
+          const uint32_t* src = v[2 * h + (j >> 3)];
+          const int i = 4 * (j & 7);
+          p[2 * j] = pack_bf16x2(__uint_as_float(src[i]) * scale * wv.x, __uint_as_float(src[i + 1]) * scale * wv.y);
+          p[2 * j + 1] =
+              pack_bf16x2(__uint_as_float(src[i + 2]) * scale * wv.z, __uint_as_float(src[i + 3]) * scale * wv.w);
         }
       } else {
 #pragma unroll
@@ -470,6 +473,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
       mbar_init(&xbars[bar_idx::SF_EMPTY + b], 1);
     }
     for (int w = 0; w < COPY_WARPS; ++w) mbar_init(&xbars[bar_idx::CP_DRAIN + w], 1);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&xbars[bar_idx::SF_LOADED + st], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -506,16 +510,18 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             break;
           }
           uint8_t* sb = smem + stage * P::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], P::STAGE_BYTES);
-          tma_load_2d(sb, &tmA, &full[stage], kt * BK_BYTES, tm * BM);
-          tma_load_2d(sb + P::A_BYTES, &tmB, &full[stage], kt * BK_BYTES, tn * BN);
+          // scales first, on their own barrier, then the code tiles
+          uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
+          mbar_arrive_expect_tx(sfl, P::SFA_BYTES + P::SFB_BYTES);
           const int64_t ka = static_cast<int64_t>(kt) * (BK / 64);
           uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
-          bulk_load(ssf, args.sfa + (tm * kunits + ka) * SF_UNIT, P::SFA_BYTES, &full[stage]);
-          bulk_load(ssf + P::SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT, P::SFB_BYTES / 2,
-                    &full[stage]);
+          bulk_load(ssf, args.sfa + (tm * kunits + ka) * SF_UNIT, P::SFA_BYTES, sfl);
+          bulk_load(ssf + P::SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT, P::SFB_BYTES / 2, sfl);
           bulk_load(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, args.sfb + ((2 * tn + 1) * kunits + ka) * SF_UNIT,
-                    P::SFB_BYTES / 2, &full[stage]);
+                    P::SFB_BYTES / 2, sfl);
+          mbar_arrive_expect_tx(&full[stage], P::A_BYTES + P::B_BYTES);
+          tma_load_2d(sb, &tmA, &full[stage], kt * BK_BYTES, tm * BM);
+          tma_load_2d(sb + P::A_BYTES, &tmB, &full[stage], kt * BK_BYTES, tn * BN);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -541,6 +547,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             phase ^= 1u;
           }
           (void)mbar_wait(&full[stage], phase, nullptr, limit, 11);
+          (void)mbar_wait(&xbars[bar_idx::SF_LOADED + stage], phase, nullptr, limit, 11);
         }
       }
     }
@@ -596,7 +603,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     // ------------------------------------------------------------------ scale copies
     if (lane == 0) {
       (void)scale_copy_loop<false, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
-          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
+          smem, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
           abort_flag, limit, 14);
     }
   } else {
@@ -677,6 +684,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
       mbar_init(&xbars[bar_idx::SF_EMPTY + b], 1);
     }
     for (int w = 0; w < COPY_WARPS; ++w) mbar_init(&xbars[bar_idx::CP_DRAIN + w], 1);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&xbars[bar_idx::SF_LOADED + st], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -720,16 +728,21 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             break;
           }
           uint8_t* sb = smem + stage * P::STAGE_BYTES;
+          // both CTAs' bytes count on the leader's barriers: scales first, on their own
+          // barrier, then the code tiles
+          uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
+          const uint32_t bar_sf = mapa_shared(smem_u32(sfl), 0);
           const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P::STAGE_BYTES);
-          tma_load_2d_pair(sb, &tmA, bar, kt * BK_BYTES, a_row);
-          tma_load_2d_pair(sb + P::A_BYTES, &tmB, bar, kt * BK_BYTES, b_row);
+          if (leader) mbar_arrive_expect_tx(sfl, 2 * (P::SFA_BYTES + P::SFB_BYTES));
           // scale units: 512 bytes = 2 rows of the 256-byte-wide scale tensor map
           uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
-          tma_load_2d_pair(ssf, &tmSFA, bar, 0, 2 * (sfa_group * kunits + 4 * kt));
-          tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar, 0, 2 * ((2 * tn) * kunits + 4 * kt));
-          tma_load_2d_pair(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, &tmSFB, bar, 0,
+          tma_load_2d_pair(ssf, &tmSFA, bar_sf, 0, 2 * (sfa_group * kunits + 4 * kt));
+          tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar_sf, 0, 2 * ((2 * tn) * kunits + 4 * kt));
+          tma_load_2d_pair(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, &tmSFB, bar_sf, 0,
                            2 * ((2 * tn + 1) * kunits + 4 * kt));
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (P::A_BYTES + P::B_BYTES));
+          tma_load_2d_pair(sb, &tmA, bar, kt * BK_BYTES, a_row);
+          tma_load_2d_pair(sb + P::A_BYTES, &tmB, bar, kt * BK_BYTES, b_row);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -753,6 +766,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             phase ^= 1u;
           }
           (void)mbar_wait(&full[stage], phase, nullptr, limit, 24);
+          (void)mbar_wait(&xbars[bar_idx::SF_LOADED + stage], phase, nullptr, limit, 24);
         }
       }
     }
@@ -807,7 +821,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     // ------------------------------------------------------------------ scale copies (leader only)
     if (leader && lane == 0) {
       (void)scale_copy_loop<true, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
-          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
+          smem, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
           abort_flag, limit, 31);
     }
   } else {

@@ -85,13 +85,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
     for (int b = 0; b < 4; ++b) {
       const uint32_t w[8] = {q[2 * b].x, q[2 * b].y, q[2 * b].z, q[2 * b].w,
                              q[2 * b + 1].x, q[2 * b + 1].y, q[2 * b + 1].z, q[2 * b + 1].w};
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[2 * i] = bf16_lo(w[i]);
-        v[2 * i + 1] = bf16_hi(w[i]);
-      }
-      const uint32_t s = quant_block16(v, G, enc, cw[2 * b], cw[2 * b + 1]);
+      const uint32_t s = quant_block16_bf16(w, G, enc, cw[2 * b], cw[2 * b + 1]);
       word |= s << (8 * b);
     }
     uint4* dst = reinterpret_cast<uint4*>(codes + r * (cols >> 1) + c * 32);
