@@ -53,6 +53,7 @@ def workload_desc(M: int) -> str:
 # capture summarised in profiles/, keyed by a hash of the GEMM's device sources: a value
 # taken on another version of the kernel is not reported.
 TRAFFIC_BY_SOURCE = {
+    "da71698da28a6a8d": 146.1e6,
 }
 
 
@@ -444,10 +445,117 @@ def cpu_baseline(M: int, rows: int = 256):
     layer.step(sample)
     dt = time.perf_counter() - t0
     fl = sum(step_flops(rows).values())
-    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{rows} random rows of the M={M} step (quantise, fp64 GEMMs, RMSNorm, SwiGLU, requant, "
-                      f"down GEMM) in {dt:.2f} s; weight packing ({layer.pack_s:.1f} s, once per model) excluded",
-            "host_threads": os.cpu_count()}
+    out = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{rows} random rows of the M={M} step (quantise, fp64 GEMMs, RMSNorm, SwiGLU, requant, "
+                     f"down GEMM) in {dt:.2f} s; weight packing ({layer.pack_s:.1f} s, once per model) excluded",
+           "host_threads": os.cpu_count()}
+    # the same oracle on one core, on a quarter of the sample
+    try:
+        from threadpoolctl import threadpool_limits
+        r1 = max(8, rows // 4)
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            layer.step(sample[:r1])
+            d1 = time.perf_counter() - t0
+        out["one_core"] = {"value": round(sum(step_flops(r1).values()) / d1 / 1e12, 6), "unit": "TFLOP/s",
+                           "sample": f"{r1} rows in {d1:.2f} s"}
+    except ImportError:  # pragma: no cover
+        pass
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# the M sweep: fused vs unfused, cold and warm L2
+# ----------------------------------------------------------------------------------
+def run_sweep(args):
+    """Fused vs unfused for M in {1024, 4096, 8192, 16384} x {QKV hd128, QKV hd256, FFN-up
+    with NVFP4 re-quantisation}. Each run is timed alone with CUDA events: cold (a 512 MB
+    buffer written before each run, primary) and warm (no scrub). 10 warm-ups, then the
+    median of --sweep-runs runs."""
+    import torch
+    import epilogues_nvfp4_quantize_b200 as ep
+    import workloads as wk
+    from epilogues_nvfp4_quantize_b200.build import build
+
+    build()
+    ep.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T = ep.NVFP4Tensor
+    scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    pk = peaks()
+    fp4_peak = pk["bf16"] * FP4_PER_BF16
+
+    def median_us(fn, cold, runs):
+        for _ in range(10):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(runs)]
+        for e0, e1 in evs:
+            if cold:
+                scrub.fill_(1)
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize(dev)
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
+
+    rows = []
+    n_launch0 = ep.launch_count()
+    for wl in wk.sweep():
+        inp = wk.make_inputs(wl)
+        a, b = inp["a"].to(dev), inp["b"].to(dev)
+        M, K, N = wl.M, wl.K, wl.N
+        A = T.empty(M, K, dev)
+        ep.nvfp4_quantize(a, A)
+        if wl.op == "rmsnorm":
+            B = T.empty(N, K, dev)
+            ep.nvfp4_quantize(b, B)
+            w = torch.from_numpy(inp["w"]).to(dev)
+            D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+            def fused():
+                ep.gemm_nvfp4_rmsnorm(A, B, w, wl.head_dim, wl.n_norm_cols, wl.eps, D)
+
+            def unfused():
+                ep.gemm_nvfp4_plain(A, B, D)
+                ep.rmsnorm_heads_bf16(D, w, wl.head_dim, wl.n_norm_cols, wl.eps, D)
+        else:
+            nh = N // 2
+            Bi, Bl = T.empty(N, K, dev), T.empty(N, K, dev)
+            ep.nvfp4_quantize(b, Bi, interleave=True)
+            ep.nvfp4_quantize(b, Bl)
+            Dq = T.empty(M, nh, dev)
+            hb = torch.empty(M, nh, dtype=torch.bfloat16, device=dev)
+            ep.gemm_nvfp4_swiglu(A, Bi, hb, None)
+            ep.nvfp4_quantize(hb, Dq)  # static scale of the re-quantised output, calibrated once
+            del hb
+            Dq2 = T(torch.empty_like(Dq.codes), torch.empty_like(Dq.sf), Dq.gscale, M, nh)
+            C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            Y = torch.empty(M, nh, dtype=torch.bfloat16, device=dev)
+
+            def fused():
+                ep.gemm_nvfp4_swiglu(A, Bi, None, Dq)
+
+            def unfused():
+                ep.gemm_nvfp4_plain(A, Bl, C)
+                ep.swiglu_bf16(C, Y)
+                ep.nvfp4_quantize(Y, Dq2, compute_amax=False)
+        r = {"workload": wl.name, "M": M, "op": wl.op, "head_dim": wl.head_dim}
+        for mode, cold in (("cold", True), ("warm", False)):
+            tf, tu = median_us(fused, cold, args.sweep_runs), median_us(unfused, cold, args.sweep_runs)
+            r[mode] = {"fused_us": round(tf, 2), "unfused_us": round(tu, 2), "speedup": round(tu / tf, 3),
+                       "fused_tflops": round(wl.flops / (tf * 1e-6) / 1e12, 1),
+                       "pct_fp4_peak": round(100.0 * wl.flops / (tf * 1e-6) / 1e12 / fp4_peak, 1)}
+        rows.append(r)
+        print(json.dumps(r), flush=True)
+        del A, a, b
+        torch.cuda.empty_cache()
+    status = ep.read_device_status()
+    print(json.dumps({"sweep": "fused vs unfused", "runs": args.sweep_runs, "warmup": 10,
+                      "fp4_peak_tflops": round(fp4_peak, 1), "peak_source": pk["source"],
+                      "launches": ep.launch_count() - n_launch0, "device_status": status}), flush=True)
+    if status != 0:
+        raise SystemExit(f"device status {status}")
 
 
 def run_reference(args):
@@ -493,6 +601,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=64, help="rows per step of the --impl reference arm")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the FFN-up kernel from an ncu capture of this kernel")
+    ap.add_argument("--sweep", action="store_true",
+                    help="fused vs unfused over M in {1024, 4096, 8192, 16384} x {QKV hd128, hd256, FFN-up}")
+    ap.add_argument("--sweep-runs", type=int, default=50)
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -501,6 +612,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_cuda(args)
 
