@@ -33,6 +33,7 @@ struct DeviceInfo {
   bool gemm_attr_set[3] = {false, false, false};
   bool pair_attr_set[3] = {false, false, false};
   int pair_clusters[3] = {0, 0, 0};
+  bool quant_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -236,25 +237,47 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
   nvfp4_status st;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
 
-  const uint16_t* xp = static_cast<const uint16_t*>(x);
-  unsigned int* amax = nullptr;
+  CUtensorMap tmX;
+  if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(cols),
+                   static_cast<uint64_t>(rows), static_cast<uint64_t>(ldx) * 2, 64,
+                   (flags & NVFP4_SWIGLU_INTERLEAVE) ? 64 : 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return NVFP4_ERR_CUDA;
+  nvfp4::QuantArgs args{};
+  args.rows = rows;
+  args.cols = cols;
+  args.interleave = (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0;
+  args.compute_amax = compute_amax;
+  args.gscale = out.gscale;
+  args.codes = static_cast<uint8_t*>(out.codes);
+  args.sf = static_cast<uint8_t*>(out.sf);
+  args.wait_limit_ns = kWaitLimitNs;
   if (compute_amax) {
-    amax = static_cast<unsigned int*>(workspace);
-    if (cudaMemsetAsync(amax, 0, sizeof(unsigned int), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
-    const int64_t units = rows * (cols / 8);
-    int64_t blocks = (units + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(info->sm_count) * 4;
-    if (blocks > cap) blocks = cap;
-    nvfp4::amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(xp, rows, cols, ldx, amax);
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    if ((st = launch_status()) != NVFP4_OK) return st;
+    args.amax_bits = static_cast<unsigned int*>(workspace);
+    args.arrived = args.amax_bits + 1;
+    if (cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned int), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
-  const int64_t rows_pad = (rows + 127) / 128 * 128;
-  const int64_t threads = rows_pad * (cols / 64);
-  const int64_t blocks = (threads + 255) / 256;
-  nvfp4::quantize_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      xp, rows, cols, ldx, (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0, amax, out.gscale,
-      static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf));
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->quant_attr_set) {
+      if (cudaFuncSetAttribute(nvfp4::quantize_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               nvfp4::qcfg::SMEM_BYTES) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      info->quant_attr_set = true;
+    }
+  }
+  const int64_t chunks = (rows + 127) / 128 * ((cols / 64 + nvfp4::qcfg::BOXES - 1) / nvfp4::qcfg::BOXES);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // the amax pass ends in a grid barrier: all CTAs resident
+  attr[0].val.cooperative = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(chunks < info->sm_count ? chunks : info->sm_count), 1, 1);
+  cfg.blockDim = dim3(nvfp4::qcfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = nvfp4::qcfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, nvfp4::quantize_stream_kernel, tmX, args) != cudaSuccess) return NVFP4_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }

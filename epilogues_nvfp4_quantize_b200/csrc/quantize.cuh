@@ -1,6 +1,7 @@
 // nvfp4_quantize: bf16 -> NVFP4 (E2M1 codes, E4M3 block scales in the tensor-core scale
-// layout, FP32 per-tensor scale). HBM-bound: an optional amax pass, then one pass that
-// reads 128 bytes and writes 36 bytes per thread.
+// layout, FP32 per-tensor scale). HBM-bound. quantize_stream_kernel is the path of
+// nvfp4_quantize; quantize_kernel (one thread per 64 values, plain loads) serves the
+// allocation-free variant, whose amax reduction runs in kernels of its own.
 #pragma once
 
 #include "ptx.cuh"
@@ -8,49 +9,8 @@
 
 namespace nvfp4 {
 
-// amax(|x|) over a rows x cols bf16 tensor, folded into *amax_bits (float bits, the
-// caller zeroes it first) with one atomicMax per block. Each thread keeps four 16-byte
-// loads in flight per iteration.
-__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                   int64_t cols, int64_t ldx,
-                                                   unsigned int* __restrict__ amax_bits) {
-  const int64_t upr = cols >> 3;  // 16-byte units per row
-  const int64_t total = rows * upr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  float m = 0.0f;
-  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u0 < total; u0 += 4 * stride) {
-    uint4 v[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t u = u0 + i * stride;
-      if (u < total) {
-        const int64_t r = u / upr, c = u - r * upr;
-        v[i] = __ldg(reinterpret_cast<const uint4*>(x + r * ldx + c * 8));
-      } else {
-        v[i] = make_uint4(0, 0, 0, 0);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t w[4] = {v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu, v[i].z & 0x7FFF7FFFu,
-                             v[i].w & 0x7FFF7FFFu};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(bf16_lo(w[k]), bf16_hi(w[k])));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ float wmax[8];
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float b = 0.0f;
-    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) b = fmaxf(b, wmax[i]);
-    if (b > 0.0f) atomicMax(amax_bits, __float_as_uint(b));
-  }
-}
-
-// Quantise rows x cols (cols % 64 == 0). One thread owns 64 adjacent values of a row:
+// Quantise rows x cols (cols % 64 == 0) with a per-tensor scale already derived (from
+// *amax_bits, or *gscale when amax_bits is null). One thread owns 64 adjacent values of a row:
 // four 16-blocks, i.e. one 4-byte scale word and 32 bytes of codes. Threads cover rows
 // padded to 128 so that the padding scale words are written as 0. With `interleave`,
 // output row 2j reads input row j and output row 2j+1 reads input row rows/2 + j.
@@ -93,6 +53,247 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
     dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
   }
   *reinterpret_cast<uint32_t*>(sf + sf_word_offset(r, 4 * c, cols >> 4)) = word;
+}
+
+// =====================================================================================
+// Streaming quantiser: one persistent CTA per SM. A producer warp moves 128-row x 64-column
+// bf16 boxes of x into a shared-memory ring with TMA (128-byte swizzle, so that the
+// consumers' 16-byte reads are free of bank conflicts); 16 consumer warps, one thread per
+// (row, 64-column group), read them. With compute_amax the CTAs first stream all of x for
+// its amax (the loads ask L2 to keep x), meet at a bounded grid barrier (cooperative
+// launch: every CTA is resident), derive G = amax / (6 * 448), then stream x again (from
+// L2 where it stayed) and quantise. A 128-row box yields one whole 512-byte scale unit of
+// each 64-column group, so the scale words of a box land in one contiguous 512 bytes.
+// =====================================================================================
+namespace qcfg {
+constexpr int CONSUMER_WARPS = 16;
+constexpr int CONSUMERS = CONSUMER_WARPS * 32;   // 512: 4 boxes x 128 rows
+constexpr int THREADS = CONSUMERS + 32;          // + TMA producer warp
+constexpr int BOX_ROWS = 128;
+constexpr int BOX_BYTES = BOX_ROWS * 128;        // 128 rows x 64 bf16
+constexpr int BOXES = CONSUMERS / BOX_ROWS;      // boxes per stage
+constexpr int STAGE_BYTES = BOXES * BOX_BYTES;   // 64 KB
+constexpr int STAGES = 3;
+constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+constexpr int SMEM_BYTES = OFF_BAR + (2 * STAGES + 2) * 8 + 16 + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+}  // namespace qcfg
+
+struct QuantArgs {
+  int64_t rows, cols;        // output rows (after the optional interleave) and columns
+  int interleave;            // output row 2j <- input row j, 2j+1 <- input row rows/2 + j
+  int compute_amax;          // 1: derive G from amax(|x|); 0: use *gscale
+  unsigned int* amax_bits;   // workspace word 0 (zeroed by the caller's stream)
+  unsigned int* arrived;     // workspace word 1: grid-barrier counter (zeroed likewise)
+  float* gscale;
+  uint8_t* codes;
+  uint8_t* sf;
+  uint64_t wait_limit_ns;
+};
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// All CTAs have arrived on *ctr (bounded wait; false on time-out).
+__device__ __forceinline__ bool grid_wait(const unsigned int* ctr, unsigned int target, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(ctr) < target) {
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// Largest magnitude of 64 bf16 values (32 packed words).
+__device__ __forceinline__ float bf16x64_amax(const uint4 (&v)[8]) {
+  uint32_t m = v[0].x;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+    for (int k = (q == 0 ? 1 : 0); k < 4; ++k) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[k]));
+  }
+  return fmaxf(fabsf(__uint_as_float(m << 16)), fabsf(__uint_as_float(m & 0xFFFF0000u)));
+}
+
+__global__ void __launch_bounds__(qcfg::THREADS, 1)
+    quantize_stream_kernel(const __grid_constant__ CUtensorMap tmX, const QuantArgs a) {
+  using namespace qcfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* red_bar = empty + STAGES;  // every consumer warp has folded its amax into s_amax
+  uint64_t* go_bar = red_bar + 1;      // G is known (after the grid barrier)
+  unsigned int* s_amax = reinterpret_cast<unsigned int*>(go_bar + 1);
+  float* s_G = reinterpret_cast<float*>(s_amax + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(s_G + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t limit = a.wait_limit_ns;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], CONSUMER_WARPS);
+    }
+    mbar_init(red_bar, CONSUMER_WARPS);
+    mbar_init(go_bar, 1);
+    *s_amax = 0u;
+    *s_G = 0.0f;
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  const int64_t num_g = a.cols >> 6;                     // 64-column groups
+  const int64_t per_rb = (num_g + BOXES - 1) / BOXES;    // chunks per 128-row block
+  const int64_t chunks = ((a.rows + 127) >> 7) * per_rb;
+  const int passes = a.compute_amax ? 2 : 1;
+
+  if (warp == CONSUMER_WARPS) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int pass = 0; ok && pass < passes; ++pass) {
+        const uint64_t pol = pass + 1 < passes ? keep : stream;
+        for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 41)) {
+            ok = false;
+            break;
+          }
+          const int64_t rb = c / per_rb;
+          const int64_t g0 = (c - rb * per_rb) * BOXES;
+          const int nb = static_cast<int>(num_g - g0 < BOXES ? num_g - g0 : BOXES);
+          mbar_arrive_expect_tx(&full[stage], nb * BOX_BYTES);
+          uint8_t* sb = smem + stage * STAGE_BYTES;
+          for (int b = 0; b < nb; ++b) {
+            const int x = static_cast<int>((g0 + b) * 64);
+            if (!a.interleave) {
+              tma_load_2d_hint(sb + b * BOX_BYTES, &tmX, &full[stage], x, static_cast<int>(rb * 128), pol);
+            } else {
+              // even output rows from the first half of x, odd ones from the second
+              tma_load_2d_hint(sb + b * BOX_BYTES, &tmX, &full[stage], x, static_cast<int>(rb * 64), pol);
+              tma_load_2d_hint(sb + b * BOX_BYTES + 64 * 128, &tmX, &full[stage], x,
+                               static_cast<int>((a.rows >> 1) + rb * 64), pol);
+            }
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // give up: wait (bounded) for the loads this thread started, then leave
+        for (int i = 0; i < STAGES && i < issued; ++i) {
+          if (--stage < 0) {
+            stage = STAGES - 1;
+            phase ^= 1u;
+          }
+          (void)mbar_wait(&full[stage], phase, nullptr, limit, 41);
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int b = threadIdx.x >> 7;   // box of the stage
+  const int i = threadIdx.x & 127;  // row of the box
+  const int sr = a.interleave ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;  // its row in shared memory
+  const uint32_t rowoff = static_cast<uint32_t>(b * BOX_BYTES + sr * 128);
+  const int sw = sr & 7;  // 128-byte swizzle: 16-byte chunk q of the row sits at q ^ sw
+  int stage = 0;
+  uint32_t phase = 0;
+  float m = 0.0f, G = 0.0f, enc = 0.0f;
+  for (int pass = 0; pass < passes; ++pass) {
+    const bool quant = pass + 1 == passes;
+    if (quant) {
+      if (a.compute_amax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) {
+          atomicMax(s_amax, __float_as_uint(m));
+          mbar_arrive(red_bar);
+        }
+        if (threadIdx.x == 0) {
+          bool good = mbar_wait(red_bar, 0, abort_flag, limit, 42);
+          if (good) {
+            if (*s_amax != 0u) atomicMax(a.amax_bits, *s_amax);
+            __threadfence();
+            atomicAdd(a.arrived, 1u);
+            good = grid_wait(a.arrived, gridDim.x, limit);
+            if (!good) {
+              *abort_flag = 1;
+              record_status(6, 43);
+            }
+          }
+          if (good) {
+            const float g = __fdiv_rn(__uint_as_float(ld_acquire_gpu(a.amax_bits)), kGlobalDiv);
+            *s_G = g;
+            if (blockIdx.x == 0) *a.gscale = g;
+          }
+          mbar_arrive(go_bar);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(go_bar, 0, abort_flag, limit, 44)) || *abort_flag) return;
+        G = *s_G;
+      } else {
+        G = *a.gscale;
+      }
+      enc = scale_encode_factor(G);
+    }
+    for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, limit, 45))) return;
+      const int64_t rb = c / per_rb;
+      const int64_t g = (c - rb * per_rb) * BOXES + b;
+      const int64_t r = rb * 128 + i;
+      if (g < num_g) {
+        uint4 v[8];
+        if (r < a.rows) {
+          const uint8_t* src = smem + stage * STAGE_BYTES + rowoff;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) v[q] = *reinterpret_cast<const uint4*>(src + ((q ^ sw) << 4));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) v[q] = make_uint4(0u, 0u, 0u, 0u);  // padding rows: zero scales
+        }
+        if (!quant) {
+          m = fmaxf(m, bf16x64_amax(v));
+        } else {
+          uint32_t cw[8];
+          uint32_t word = 0;
+#pragma unroll
+          for (int blk = 0; blk < 4; ++blk) {
+            const uint32_t w[8] = {v[2 * blk].x,     v[2 * blk].y,     v[2 * blk].z,     v[2 * blk].w,
+                                   v[2 * blk + 1].x, v[2 * blk + 1].y, v[2 * blk + 1].z, v[2 * blk + 1].w};
+            word |= quant_block16_bf16(w, G, enc, cw[2 * blk], cw[2 * blk + 1]) << (8 * blk);
+          }
+          if (r < a.rows) {
+            uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + g * 32);
+            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          }
+          *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(r, 4 * g, a.cols >> 4)) = word;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
 }
 
 }  // namespace nvfp4

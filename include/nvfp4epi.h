@@ -84,7 +84,11 @@ int64_t nvfp4_quantize_workspace_bytes(void);
  * Quantise a bf16 tensor x (rows x cols, leading dimension ldx elements) to NVFP4.
  *   compute_amax = 1: G = amax(|x|) / (6 * 448) is computed on the device and written to
  *                     *out.gscale; `workspace` must hold
- *                     nvfp4_quantize_workspace_bytes() bytes (contents on entry ignored).
+ *                     nvfp4_quantize_workspace_bytes() bytes, 4-byte aligned (contents on
+ *                     entry ignored: the call clears it on `stream`). It holds the amax and
+ *                     the counter of a grid barrier, so calls that share a workspace must
+ *                     not overlap. The kernel is a cooperative launch (one CTA per SM); it
+ *                     reads x twice, the second time mostly from L2.
  *   compute_amax = 0: *out.gscale is used as given (static scale, must be > 0 and finite);
  *                     workspace may be NULL.
  * Per block of 16, in IEEE float32: s = E4M3_rn_satfinite(amax_b * (1 / (6 G))) (s = 0

@@ -38,6 +38,19 @@ def test_quantize_interleaved_weight():
     _check_bitwise(w, t, interleave=True)
 
 
+@pytest.mark.parametrize("nh,cols", [(100, 320), (1000, 64)])
+def test_quantize_interleaved_ragged(nh, cols):
+    # 2*nh rows: the halves start off a 64-row boundary and the last 128-row block is partial
+    w = wk.weights(2 * nh, cols, 1 / np.sqrt(cols), seed=nh)
+    _check_bitwise(w, quantize_gpu(w, interleave=True), interleave=True)
+
+
+def test_quantize_static_scale_many_blocks_per_cta():
+    x = wk.activations(4000, 1984, 2, seed=21)  # 32 x 8 chunks of 128 rows x 256 columns
+    G = np.float32(np.abs(x.float().numpy()).max() / 2688)
+    _check_bitwise(x, quantize_gpu(x, G=G), G_static=G)
+
+
 def test_quantize_static_scale_including_saturation():
     x = wk.activations(256, 512, 2, seed=9)
     G = np.float32(np.abs(x.float().numpy()).max() / 2688 / 4)  # too small: saturates
