@@ -237,14 +237,22 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
   nvfp4_status st;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
 
+  // stage shape: G boxes of R rows x 64 columns, G * R = 512 (G = 16 from 1024 columns up)
+  const int64_t num_g = cols / 64;
+  int G = 16;
+  while (G > 1 && G > num_g) G >>= 1;
+  const int R = G >= 2 ? 512 / G : 256;
+  const bool inter = (flags & NVFP4_SWIGLU_INTERLEAVE) != 0;
   CUtensorMap tmX;
   if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(cols),
                    static_cast<uint64_t>(rows), static_cast<uint64_t>(ldx) * 2, 64,
-                   (flags & NVFP4_SWIGLU_INTERLEAVE) ? 64 : 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint32_t>(inter ? R / 2 : R), CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ERR_CUDA;
   nvfp4::QuantArgs args{};
   args.rows = rows;
   args.cols = cols;
+  args.box_rows = R;
+  args.boxes = G;
   args.interleave = (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0;
   args.compute_amax = compute_amax;
   args.gscale = out.gscale;
@@ -265,7 +273,8 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
       info->quant_attr_set = true;
     }
   }
-  const int64_t chunks = (rows + 127) / 128 * ((cols / 64 + nvfp4::qcfg::BOXES - 1) / nvfp4::qcfg::BOXES);
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t chunks = (rows_pad + R - 1) / R * ((num_g + G - 1) / G);
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];

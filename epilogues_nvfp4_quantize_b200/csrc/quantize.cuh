@@ -56,23 +56,20 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
 }
 
 // =====================================================================================
-// Streaming quantiser: one persistent CTA per SM. A producer warp moves 128-row x 64-column
-// bf16 boxes of x into a shared-memory ring with TMA (128-byte swizzle, so that the
-// consumers' 16-byte reads are free of bank conflicts); 16 consumer warps, one thread per
-// (row, 64-column group), read them. With compute_amax the CTAs first stream all of x for
-// its amax (the loads ask L2 to keep x), meet at a bounded grid barrier (cooperative
-// launch: every CTA is resident), derive G = amax / (6 * 448), then stream x again (from
-// L2 where it stayed) and quantise. A 128-row box yields one whole 512-byte scale unit of
-// each 64-column group, so the scale words of a box land in one contiguous 512 bytes.
+// Streaming quantiser: one persistent CTA per SM. A producer warp moves stages of
+// R rows x 64G columns of x (G boxes of R rows x 64 bf16, G x R = 512; G = 16 when x has at
+// least 1024 columns, so a stage reads 2 KB runs of 32 rows) into a shared-memory ring with
+// TMA. The 128-byte swizzle keeps the consumers' 16-byte reads free of bank conflicts. 16
+// consumer warps, one thread per (row, 64-column group), read them. With compute_amax the
+// CTAs first stream all of x for its amax (the loads ask L2 to keep x), meet at a bounded
+// grid barrier (cooperative launch: every CTA is resident), derive G = amax / (6 * 448),
+// then stream x again (from L2 where it stayed) and quantise.
 // =====================================================================================
 namespace qcfg {
 constexpr int CONSUMER_WARPS = 16;
 constexpr int CONSUMERS = CONSUMER_WARPS * 32;   // 512: 4 boxes x 128 rows
 constexpr int THREADS = CONSUMERS + 32;          // + TMA producer warp
-constexpr int BOX_ROWS = 128;
-constexpr int BOX_BYTES = BOX_ROWS * 128;        // 128 rows x 64 bf16
-constexpr int BOXES = CONSUMERS / BOX_ROWS;      // boxes per stage
-constexpr int STAGE_BYTES = BOXES * BOX_BYTES;   // 64 KB
+constexpr int STAGE_BYTES = CONSUMERS * 128;     // 64 KB: 512 units of 64 bf16
 constexpr int STAGES = 3;
 constexpr int OFF_BAR = STAGES * STAGE_BYTES;
 constexpr int SMEM_BYTES = OFF_BAR + (2 * STAGES + 2) * 8 + 16 + 1024;  // + alignment slack
@@ -81,6 +78,8 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 struct QuantArgs {
   int64_t rows, cols;        // output rows (after the optional interleave) and columns
+  int box_rows;              // R: rows per stage (32 .. 256, a power of two)
+  int boxes;                 // G: 64-column boxes per stage (R * G <= 512)
   int interleave;            // output row 2j <- input row j, 2j+1 <- input row rows/2 + j
   int compute_amax;          // 1: derive G from amax(|x|); 0: use *gscale
   unsigned int* amax_bits;   // workspace word 0 (zeroed by the caller's stream)
@@ -149,9 +148,11 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
   }
   __syncthreads();
 
-  const int64_t num_g = a.cols >> 6;                     // 64-column groups
-  const int64_t per_rb = (num_g + BOXES - 1) / BOXES;    // chunks per 128-row block
-  const int64_t chunks = ((a.rows + 127) >> 7) * per_rb;
+  const int R = a.box_rows, NB = a.boxes;
+  const int64_t num_g = a.cols >> 6;                       // 64-column groups
+  const int64_t rows_pad = (a.rows + 127) & ~int64_t(127);  // rows that carry scale words
+  const int64_t per_rs = (num_g + NB - 1) / NB;             // chunks per R-row slab
+  const int64_t chunks = ((rows_pad + R - 1) / R) * per_rs;
   const int passes = a.compute_amax ? 2 : 1;
 
   if (warp == CONSUMER_WARPS) {
@@ -170,20 +171,20 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
             ok = false;
             break;
           }
-          const int64_t rb = c / per_rb;
-          const int64_t g0 = (c - rb * per_rb) * BOXES;
-          const int nb = static_cast<int>(num_g - g0 < BOXES ? num_g - g0 : BOXES);
-          mbar_arrive_expect_tx(&full[stage], nb * BOX_BYTES);
+          const int64_t rs = c / per_rs;
+          const int64_t g0 = (c - rs * per_rs) * NB;
+          const int nb = static_cast<int>(num_g - g0 < NB ? num_g - g0 : NB);
+          mbar_arrive_expect_tx(&full[stage], nb * R * 128);
           uint8_t* sb = smem + stage * STAGE_BYTES;
           for (int b = 0; b < nb; ++b) {
             const int x = static_cast<int>((g0 + b) * 64);
             if (!a.interleave) {
-              tma_load_2d_hint(sb + b * BOX_BYTES, &tmX, &full[stage], x, static_cast<int>(rb * 128), pol);
+              tma_load_2d_hint(sb + b * R * 128, &tmX, &full[stage], x, static_cast<int>(rs * R), pol);
             } else {
               // even output rows from the first half of x, odd ones from the second
-              tma_load_2d_hint(sb + b * BOX_BYTES, &tmX, &full[stage], x, static_cast<int>(rb * 64), pol);
-              tma_load_2d_hint(sb + b * BOX_BYTES + 64 * 128, &tmX, &full[stage], x,
-                               static_cast<int>((a.rows >> 1) + rb * 64), pol);
+              tma_load_2d_hint(sb + b * R * 128, &tmX, &full[stage], x, static_cast<int>(rs * (R / 2)), pol);
+              tma_load_2d_hint(sb + b * R * 128 + (R / 2) * 128, &tmX, &full[stage], x,
+                               static_cast<int>((a.rows >> 1) + rs * (R / 2)), pol);
             }
           }
           ++issued;
@@ -208,10 +209,10 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
   }
 
   // ------------------------------------------------------------------ consumers
-  const int b = threadIdx.x >> 7;   // box of the stage
-  const int i = threadIdx.x & 127;  // row of the box
-  const int sr = a.interleave ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;  // its row in shared memory
-  const uint32_t rowoff = static_cast<uint32_t>(b * BOX_BYTES + sr * 128);
+  const int b = threadIdx.x / R;  // box of the stage (threads past R * NB stay idle)
+  const int i = threadIdx.x % R;  // row of the box
+  const int sr = a.interleave ? ((i & 1) ? R / 2 + (i >> 1) : (i >> 1)) : i;  // its row in shared memory
+  const uint32_t rowoff = static_cast<uint32_t>(b * R * 128 + sr * 128);
   const int sw = sr & 7;  // 128-byte swizzle: 16-byte chunk q of the row sits at q ^ sw
   int stage = 0;
   uint32_t phase = 0;
@@ -254,10 +255,10 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
     }
     for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
       if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, limit, 45))) return;
-      const int64_t rb = c / per_rb;
-      const int64_t g = (c - rb * per_rb) * BOXES + b;
-      const int64_t r = rb * 128 + i;
-      if (g < num_g) {
+      const int64_t rs = c / per_rs;
+      const int64_t g = (c - rs * per_rs) * NB + b;
+      const int64_t r = rs * R + i;
+      if (b < NB && g < num_g && r < rows_pad) {
         uint4 v[8];
         if (r < a.rows) {
           const uint8_t* src = smem + stage * STAGE_BYTES + rowoff;
