@@ -357,6 +357,27 @@ def run_cuda(args):
         del layer.c_up, layer.y_up
         torch.cuda.empty_cache()
 
+    # ---- fake quantisation (quantization-aware distillation forward), HBM-bound
+    if not args.no_unfused:
+        y_fq = torch.empty_like(layer.x)
+        g_fq = torch.empty(1, dtype=torch.float32, device=dev)
+        barrier()
+        t_fq = time_loop(lambda: ep.nvfp4_fake_quantize(layer.x, y=y_fq, gscale=g_fq, workspace=layer.ws),
+                         args.cmp_steps, 3, torch)
+        t_fq_static = time_loop(lambda: ep.nvfp4_fake_quantize(layer.x, y=y_fq, gscale=g_fq, compute_amax=False),
+                                args.cmp_steps, 3, torch)
+        fq_bytes = layer.x.numel() * 4  # read x, write y (bf16)
+        result["fake_quant"] = {
+            "shape": list(layer.x.shape),
+            "amax_us": round(t_fq * 1e3, 2), "static_us": round(t_fq_static * 1e3, 2),
+            "amax_gbs": round(fq_bytes / (t_fq * 1e-3) / 1e9, 1),
+            "static_gbs": round(fq_bytes / (t_fq_static * 1e-3) / 1e9, 1),
+            "hbm_peak_gbs": pk["hbm_gbs"],
+            "note": "algorithmic bytes = 2 B read + 2 B written per element; with amax the kernel "
+                    "reads x twice (the second time mostly from L2)",
+        }
+        del y_fq
+
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
         x_host = layer.x.cpu().pin_memory()

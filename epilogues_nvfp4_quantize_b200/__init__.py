@@ -6,12 +6,14 @@ The Python names mirror the C entry points of include/nvfp4epi.h.
 from ._lib import (  # noqa: F401
     EXPORTS,
     LIB_PATH,
+    FakeQuantizeSTE,
     NVFP4Tensor,
     gemm_nvfp4_plain,
     gemm_nvfp4_rmsnorm,
     gemm_nvfp4_swiglu,
     launch_count,
     load,
+    nvfp4_fake_quantize,
     nvfp4_quantize,
     nvfp4_quantize_noalloc,
     quantize_workspace_bytes,

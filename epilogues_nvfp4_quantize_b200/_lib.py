@@ -24,7 +24,7 @@ EXPORTS = (
     "gemm_nvfp4_plain", "gemm_nvfp4_rmsnorm", "gemm_nvfp4_swiglu",
     "rmsnorm_heads_bf16", "swiglu_bf16", "nvfp4_status_string",
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
-    "nvfp4_quantize_noalloc",
+    "nvfp4_quantize_noalloc", "nvfp4_fake_quantize",
 )
 
 
@@ -59,6 +59,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_selftest_bounded_wait": (i32, [i64, vp]),
         "nvfp4_launch_count": (i64, []),
         "nvfp4_quantize_noalloc": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
+        "nvfp4_fake_quantize": (i32, [vp, i64, i64, i64, i32, vp, vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -186,6 +187,42 @@ def nvfp4_quantize_noalloc(x: torch.Tensor, out: NVFP4Tensor, interleave: bool =
                                          SWIGLU_INTERLEAVE if interleave else 0, out.c(), _stream(stream)),
            "nvfp4_quantize_noalloc")
     return out
+
+
+def nvfp4_fake_quantize(x: torch.Tensor, y: Optional[torch.Tensor] = None, gscale: Optional[torch.Tensor] = None,
+                        compute_amax: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Quantise-dequantise a 2-D bf16 CUDA tensor through NVFP4 (see nvfp4_fake_quantize in
+    the header). Returns (y, gscale); gscale is a 1-element float32 device tensor, written
+    when compute_amax, read otherwise."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    if y is None:
+        y = torch.empty_like(x, memory_format=torch.contiguous_format)
+    py, ldy = _out2d(y)
+    if gscale is None:
+        if not compute_amax:
+            raise ValueError("a static scale needs gscale")
+        gscale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    if compute_amax and workspace is None:
+        workspace = torch.empty((quantize_workspace_bytes(),), dtype=torch.uint8, device=x.device)
+    _check(load().nvfp4_fake_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), int(compute_amax),
+                                      gscale.data_ptr(), py, ldy, _ptr(workspace), _stream(stream)),
+           "nvfp4_fake_quantize")
+    return y, gscale
+
+
+class FakeQuantizeSTE(torch.autograd.Function):
+    """y = nvfp4_fake_quantize(x) forward; identity backward (straight-through estimator:
+    the rounding is left out of the gradient, which flows at full precision)."""
+
+    @staticmethod
+    def forward(ctx, x, gscale=None, compute_amax=True):
+        y, _ = nvfp4_fake_quantize(x.contiguous(), gscale=gscale, compute_amax=compute_amax)
+        return y
+
+    @staticmethod
+    def backward(ctx, grad_y):
+        return grad_y, None, None
 
 
 def read_device_status(stream=None) -> int:

@@ -210,39 +210,17 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
 
 }  // namespace
 
-NVFP4_API int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols) {
-  if (rows < 0 || cols < 0) return -1;
-  return ((rows + 127) / 128) * 128 * ((cols / 16 + 3) / 4) * 4;
-}
-
-NVFP4_API int64_t nvfp4_quantize_workspace_bytes(void) { return 16; }
-
-NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int compute_amax,
-                                      int flags, nvfp4_tensor out, void* workspace, cudaStream_t stream) {
-  if (x == nullptr || out.codes == nullptr || out.sf == nullptr || out.gscale == nullptr)
-    return NVFP4_ERR_INVALID_ARG;
-  if (compute_amax != 0 && compute_amax != 1) return NVFP4_ERR_INVALID_ARG;
-  if (compute_amax && workspace == nullptr) return NVFP4_ERR_INVALID_ARG;
-  if (flags & ~NVFP4_SWIGLU_INTERLEAVE) return NVFP4_ERR_INVALID_ARG;
-  if (out.rows != rows || out.cols != cols) return NVFP4_ERR_INVALID_ARG;
-  if (rows <= 0 || cols <= 0 || cols % 64 != 0 || ldx < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if ((flags & NVFP4_SWIGLU_INTERLEAVE) && (rows % 2) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (rows > (1ll << 31) || cols > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(x) || (ldx % 8) != 0 || !aligned16(out.codes) ||
-      (reinterpret_cast<uintptr_t>(out.sf) & 3u) != 0 ||
-      (compute_amax && (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0))
-    return NVFP4_ERR_MISALIGNED;
-  int dev;
-  DeviceInfo* info;
-  nvfp4_status st;
-  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
-
+// Launch of the streaming quantiser (quantize.cuh) for nvfp4_quantize and
+// nvfp4_fake_quantize: codes/sf and/or the dequantised bf16 y.
+static nvfp4_status launch_quantize_stream(DeviceInfo* info, const void* x, int64_t rows, int64_t cols,
+                                           int64_t ldx, int compute_amax, bool inter, float* gscale,
+                                           uint8_t* codes, uint8_t* sf, uint16_t* y, int64_t ldy, void* workspace,
+                                           cudaStream_t stream) {
   // stage shape: G boxes of R rows x 64 columns, G * R = 512 (G = 16 from 1024 columns up)
   const int64_t num_g = cols / 64;
   int G = 16;
   while (G > 1 && G > num_g) G >>= 1;
   const int R = G >= 2 ? 512 / G : 256;
-  const bool inter = (flags & NVFP4_SWIGLU_INTERLEAVE) != 0;
   CUtensorMap tmX;
   if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(cols),
                    static_cast<uint64_t>(rows), static_cast<uint64_t>(ldx) * 2, 64,
@@ -253,11 +231,13 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
   args.cols = cols;
   args.box_rows = R;
   args.boxes = G;
-  args.interleave = (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0;
+  args.interleave = inter ? 1 : 0;
   args.compute_amax = compute_amax;
-  args.gscale = out.gscale;
-  args.codes = static_cast<uint8_t*>(out.codes);
-  args.sf = static_cast<uint8_t*>(out.sf);
+  args.gscale = gscale;
+  args.codes = codes;
+  args.sf = sf;
+  args.y = y;
+  args.ldy = ldy;
   args.wait_limit_ns = kWaitLimitNs;
   if (compute_amax) {
     args.amax_bits = static_cast<unsigned int*>(workspace);
@@ -289,6 +269,58 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
   if (cudaLaunchKernelEx(&cfg, nvfp4::quantize_stream_kernel, tmX, args) != cudaSuccess) return NVFP4_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
+}
+
+NVFP4_API int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return -1;
+  return ((rows + 127) / 128) * 128 * ((cols / 16 + 3) / 4) * 4;
+}
+
+NVFP4_API int64_t nvfp4_quantize_workspace_bytes(void) { return 16; }
+
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int compute_amax,
+                                      int flags, nvfp4_tensor out, void* workspace, cudaStream_t stream) {
+  if (x == nullptr || out.codes == nullptr || out.sf == nullptr || out.gscale == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (compute_amax != 0 && compute_amax != 1) return NVFP4_ERR_INVALID_ARG;
+  if (compute_amax && workspace == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~NVFP4_SWIGLU_INTERLEAVE) return NVFP4_ERR_INVALID_ARG;
+  if (out.rows != rows || out.cols != cols) return NVFP4_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || cols % 64 != 0 || ldx < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((flags & NVFP4_SWIGLU_INTERLEAVE) && (rows % 2) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > (1ll << 31) || cols > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx % 8) != 0 || !aligned16(out.codes) ||
+      (reinterpret_cast<uintptr_t>(out.sf) & 3u) != 0 ||
+      (compute_amax && (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+
+  return launch_quantize_stream(info, x, rows, cols, ldx, compute_amax, (flags & NVFP4_SWIGLU_INTERLEAVE) != 0,
+                                out.gscale, static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf), nullptr,
+                                0, workspace, stream);
+}
+
+NVFP4_API nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int compute_amax,
+                                           float* gscale, void* y, int64_t ldy, void* workspace,
+                                           cudaStream_t stream) {
+  if (x == nullptr || y == nullptr || gscale == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (compute_amax != 0 && compute_amax != 1) return NVFP4_ERR_INVALID_ARG;
+  if (compute_amax && workspace == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || cols % 64 != 0 || ldx < cols || ldy < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > (1ll << 31) || cols > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx % 8) != 0 || !aligned16(y) || (ldy % 8) != 0 ||
+      (reinterpret_cast<uintptr_t>(gscale) & 3u) != 0 ||
+      (compute_amax && (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  return launch_quantize_stream(info, x, rows, cols, ldx, compute_amax, false, gscale, nullptr, nullptr,
+                                static_cast<uint16_t*>(y), ldy, workspace, stream);
 }
 
 NVFP4_API nvfp4_status gemm_nvfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,

@@ -85,10 +85,38 @@ struct QuantArgs {
   unsigned int* amax_bits;   // workspace word 0 (zeroed by the caller's stream)
   unsigned int* arrived;     // workspace word 1: grid-barrier counter (zeroed likewise)
   float* gscale;
-  uint8_t* codes;
+  uint8_t* codes;            // codes and scales (or null: fake quantisation only)
   uint8_t* sf;
+  uint16_t* y;               // quantise-dequantise output in bf16 (or null)
+  int64_t ldy;
   uint64_t wait_limit_ns;
 };
+
+// Dequantised bf16 values of one 16-block: bf16(fp32(e2m1(q) * e4m3(s)) * G). The
+// level-scale products are exact in f16 (at most 2 + 4 significant bits, magnitudes from
+// 2^-10 to 2688), so they are formed two at a time with one f16x2 multiply.
+__device__ __forceinline__ void dequant_block16_bf16(uint32_t c_lo, uint32_t c_hi, uint32_t s, float G,
+                                                     uint32_t (&out)[8]) {
+  uint32_t sv2;
+  asm("{\n\t.reg .b16 h;\n\tcvt.rn.f16x2.e4m3x2 %0, %1;\n\tmov.b32 {h, _}, %0;\n\tmov.b32 %0, {h, h};\n\t}"
+      : "=r"(sv2)
+      : "h"(static_cast<uint16_t>(s & 0xFFu)));
+  const uint32_t cw[2] = {c_lo, c_hi};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t lv2, p2;
+      asm("{\n\t.reg .b8 c;\n\tcvt.u8.u32 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+          : "=r"(lv2)
+          : "r"((cw[h] >> (8 * k)) & 0xFFu));
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p2) : "r"(lv2), "r"(sv2));
+      const float lo = __half2float(__ushort_as_half(static_cast<unsigned short>(p2 & 0xFFFFu)));
+      const float hi = __half2float(__ushort_as_half(static_cast<unsigned short>(p2 >> 16)));
+      out[4 * h + k] = pack_bf16x2(__fmul_rn(lo, G), __fmul_rn(hi, G));
+    }
+  }
+}
 
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
   unsigned int v;
@@ -279,12 +307,24 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
                                    v[2 * blk + 1].x, v[2 * blk + 1].y, v[2 * blk + 1].z, v[2 * blk + 1].w};
             word |= quant_block16_bf16(w, G, enc, cw[2 * blk], cw[2 * blk + 1]) << (8 * blk);
           }
-          if (r < a.rows) {
-            uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + g * 32);
-            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          if (a.codes != nullptr) {
+            if (r < a.rows) {
+              uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + g * 32);
+              dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+              dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            }
+            *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(r, 4 * g, a.cols >> 4)) = word;
           }
-          *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(r, 4 * g, a.cols >> 4)) = word;
+          if (a.y != nullptr && r < a.rows) {
+            uint4* dst = reinterpret_cast<uint4*>(a.y + r * a.ldy + g * 64);
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+              uint32_t o[8];
+              dequant_block16_bf16(cw[2 * blk], cw[2 * blk + 1], (word >> (8 * blk)) & 0xFFu, G, o);
+              dst[2 * blk] = make_uint4(o[0], o[1], o[2], o[3]);
+              dst[2 * blk + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+          }
         }
       }
       __syncwarp();

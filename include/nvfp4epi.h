@@ -106,6 +106,24 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
                             void* workspace, cudaStream_t stream);
 
 /*
+ * Fake quantisation (quantise-dequantise) for quantization-aware distillation ("Serving
+ * sub-second Ideogram v4 without quality loss", section "Quantization-aware distillation":
+ * the forward pass carries the FP4 rounding noise, the backward pass lets the gradient
+ * through unchanged, the straight-through estimator, which needs no kernel).
+ * y (rows x cols bf16, leading dimension ldy) = bf16(fp32(e2m1(q) * e4m3(s)) * G), where
+ * q, s, G are exactly what nvfp4_quantize would produce for x (the level-scale product is
+ * exact; the product with G is one fp32 rounding, then round to nearest even bf16).
+ *   compute_amax = 1: G = amax(|x|) / (6 * 448) is derived on the device and written to
+ *                     *gscale; `workspace` as for nvfp4_quantize.
+ *   compute_amax = 0: *gscale is used as given (static scale); workspace may be NULL.
+ * Rules: rows >= 1, cols % 64 == 0, ldx >= cols, ldy >= cols, x, y, ldx*2 and ldy*2
+ *        bytes 16-byte aligned, gscale 4-byte aligned. y may not overlap x.
+ */
+nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                 int compute_amax, float* gscale, void* y, int64_t ldy,
+                                 void* workspace, cudaStream_t stream);
+
+/*
  * D (M x N bf16, leading dimension ldd) = bf16(G_A * G_B * sum_k A[m,k] * B[n,k]) with
  * A (M x K) and B (N x K) NVFP4, both K-contiguous.
  * Rules: M % 128 == 0, N % 256 == 0, K % 256 == 0, A.cols == B.cols == K,

@@ -186,6 +186,21 @@ def dequantize(codes, scales, G) -> np.ndarray:
     return vals.reshape(rows, cols)
 
 
+def fake_quantize(x, G=None):
+    """Quantise-dequantise ("fake quantisation" of quantisation-aware distillation, page
+    "Serving sub-second Ideogram v4 without quality loss", section on quantization-aware
+    distillation): the forward pass sees the FP4 rounding noise. Returns (y, G) with
+    y = bf16(fp32(e2m1(q) * e4m3(s)) * fp32 G): the level-scale product is exact in fp32,
+    the product with G is one fp32 rounding, the result is rounded to bf16 (RNE).
+    The backward pass (straight-through estimator) is the identity and needs no oracle."""
+    q, s, G = quantize(x, G)
+    rows, cols = q.shape
+    ls = (_E2M1_TABLE[q & 0xF].reshape(rows, cols // BLOCK, BLOCK)
+          * _E4M3_TABLE[np.asarray(s)][:, :, None]).reshape(rows, cols)
+    y32 = ls.astype(np.float32) * np.float32(G)
+    return bf16_round(y32.astype(np.float64)), G
+
+
 # ----------------------------------------------------------------------------------
 # Storage layouts read by the tensor cores (an independent statement of the byte
 # layout, used to read GPU buffers and to build GPU inputs in tests)

@@ -117,3 +117,52 @@ def test_scale_and_code_packing_roundtrip():
     assert p.shape == (5, 32)
     assert np.array_equal(p[:, 0] & 0xF, c[:, 0]) and np.array_equal(p[:, 0] >> 4, c[:, 1])
     assert np.array_equal(o.unpack_codes(p), c)
+
+
+# ---- fake quantisation (quantise-dequantise) -------------------------------------
+
+def _representable(rows, cols, G, seed):
+    """Blocks whose largest magnitude is 6 * e4m3(s) * G: every element is level * scale * G,
+    exactly, for a power-of-two G."""
+    rng = np.random.default_rng(seed)
+    lv = o.e2m1_decode(np.arange(16))
+    q = rng.integers(0, 16, size=(rows, cols))
+    q[:, ::16] = 7  # the block maximum (+6)
+    s = rng.integers(0x20, 0x7E, size=(rows, cols // 16))  # normal E4M3 scales
+    x = lv[q] * np.repeat(o.e4m3_decode(s), 16, axis=1) * float(G)
+    return x.astype(np.float32)
+
+
+def test_fake_quantize_returns_representable_values_unchanged():
+    G = np.float32(2.0 ** -7)
+    x = _representable(64, 256, G, seed=1)
+    y, G2 = o.fake_quantize(x, G)
+    assert G2 == G
+    # level * scale * G has at most 7 significant bits here, so bf16 holds it exactly
+    assert np.array_equal(y, x.astype(np.float64))
+
+
+def test_fake_quantize_is_idempotent_at_power_of_two_scale():
+    G = np.float32(2.0 ** -9)
+    x = _rand(128, 512, seed=8, outliers=2)
+    y, _ = o.fake_quantize(x, G)
+    y2, _ = o.fake_quantize(y.astype(np.float32), G)
+    assert np.array_equal(y2, y)
+
+
+def test_fake_quantize_is_odd_and_close_to_the_exact_dequantisation():
+    x = _rand(64, 512, seed=9, outliers=3)
+    y, G = o.fake_quantize(x)
+    yn, Gn = o.fake_quantize(-x)
+    assert Gn == G and np.array_equal(yn, -y)
+    q, s, _ = o.quantize(x)
+    exact = o.dequantize(q, s, G)  # float64, no rounding
+    # one fp32 and one bf16 rounding: within 2^-8 relative (plus fp32 underflow slack)
+    assert np.all(np.abs(y - exact) <= 2.0 ** -8 * np.abs(exact) + 1e-30)
+    # and the fake-quantised tensor stays within half a level step of x (FP4-sized error)
+    assert np.abs(y - x).max() <= 0.5 * 2.0 * 448 * float(G) * 1.01
+
+
+def test_fake_quantize_of_zero_is_zero():
+    y, G = o.fake_quantize(np.zeros((128, 64), np.float32))
+    assert G == 0 and not y.any()
