@@ -357,6 +357,28 @@ def run_cuda(args):
         del layer.c_up, layer.y_up
         torch.cuda.empty_cache()
 
+    # ---- pointwise epilogues (bias, ReLU, cast, NVFP4 output) on the FFN-down GEMM
+    if not args.no_unfused:
+        bias = torch.randn(K_IN, device=dev, dtype=torch.float32) * 0.01
+        d32 = torch.empty(M, K_IN, dtype=torch.float32, device=dev)
+        dq = ep.NVFP4Tensor.empty(M, K_IN, dev)
+        dq.gscale.fill_(float(layer.out.float().abs().max().item()) / 2688)
+        barrier()
+        cases = {
+            "plain_bf16": lambda: ep.gemm_nvfp4_plain(layer.h, layer.Wdown, layer.out),
+            "bias_relu_bf16": lambda: ep.gemm_nvfp4_pointwise(layer.h, layer.Wdown, layer.out, bias=bias, relu=True),
+            "bias_f32": lambda: ep.gemm_nvfp4_pointwise(layer.h, layer.Wdown, d32, bias=bias),
+            "bias_relu_nvfp4_only": lambda: ep.gemm_nvfp4_pointwise(layer.h, layer.Wdown, None, bias=bias, relu=True,
+                                                                   Dq=dq),
+        }
+        pw = {}
+        for name, fn in cases.items():
+            t = time_loop(fn, args.cmp_steps, 3, torch)
+            pw[name] = {"us": round(t * 1e3, 1), "tflops": round(flops["down"] / (t * 1e-3) / 1e12, 1)}
+        pw["shape"] = f"M={M} K={K_DOWN} N={K_IN} (FFN-down)"
+        result["pointwise"] = pw
+        del d32, dq
+
     # ---- fake quantisation (quantization-aware distillation forward), HBM-bound
     if not args.no_unfused:
         y_fq = torch.empty_like(layer.x)

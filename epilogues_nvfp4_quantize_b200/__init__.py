@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     FakeQuantizeSTE,
     NVFP4Tensor,
     gemm_nvfp4_plain,
+    gemm_nvfp4_pointwise,
     gemm_nvfp4_rmsnorm,
     gemm_nvfp4_swiglu,
     launch_count,

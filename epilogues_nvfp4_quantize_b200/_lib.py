@@ -24,7 +24,7 @@ EXPORTS = (
     "gemm_nvfp4_plain", "gemm_nvfp4_rmsnorm", "gemm_nvfp4_swiglu",
     "rmsnorm_heads_bf16", "swiglu_bf16", "nvfp4_status_string",
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
-    "nvfp4_quantize_noalloc", "nvfp4_fake_quantize",
+    "nvfp4_quantize_noalloc", "nvfp4_fake_quantize", "gemm_nvfp4_pointwise",
 )
 
 
@@ -60,6 +60,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_launch_count": (i64, []),
         "nvfp4_quantize_noalloc": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
         "nvfp4_fake_quantize": (i32, [vp, i64, i64, i64, i32, vp, vp, i64, vp, vp]),
+        "gemm_nvfp4_pointwise": (i32, [_Tensor, _Tensor, vp, i32, i32, vp, i64, ctypes.POINTER(_Tensor), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -154,6 +155,29 @@ def gemm_nvfp4_swiglu(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tensor] 
     p, ld = _out2d(D)
     dq = ctypes.pointer(Dq.c()) if Dq is not None else None
     _check(load().gemm_nvfp4_swiglu(A.c(), B.c(), p, ld, dq, _stream(stream)), "gemm_nvfp4_swiglu")
+    return D, Dq
+
+
+ACT_NONE, ACT_RELU = 0, 1
+_OUT_KIND = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+
+
+def gemm_nvfp4_pointwise(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tensor] = None,
+                         bias: Optional[torch.Tensor] = None, relu: bool = False,
+                         Dq: Optional[NVFP4Tensor] = None, stream=None):
+    """D = cast(act(G_A G_B acc + bias)) in D's dtype (bf16, f16 or f32) and/or Dq = NVFP4 of
+    bf16 of it with Dq's static scale (see gemm_nvfp4_pointwise in the header)."""
+    if bias is not None and (bias.dtype != torch.float32 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous float32 tensor")
+    if D is not None:
+        if D.dtype not in _OUT_KIND or D.dim() != 2 or D.stride(1) != 1:
+            raise ValueError("D must be a 2-D bf16, f16 or f32 tensor with unit column stride")
+        p, ld, kind = D.data_ptr(), D.stride(0), _OUT_KIND[D.dtype]
+    else:
+        p, ld, kind = None, 0, 0
+    dq = ctypes.pointer(Dq.c()) if Dq is not None else None
+    _check(load().gemm_nvfp4_pointwise(A.c(), B.c(), _ptr(bias), ACT_RELU if relu else ACT_NONE, kind, p, ld, dq,
+                                       _stream(stream)), "gemm_nvfp4_pointwise")
     return D, Dq
 
 

@@ -126,5 +126,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
   return *reinterpret_cast<const uint32_t*>(&p);
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 p = __floats2half2_rn(lo, hi);  // .x = lo (low half), .y = hi
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
 
 }  // namespace nvfp4

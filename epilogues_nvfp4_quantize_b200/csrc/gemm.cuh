@@ -31,6 +31,10 @@
 //            warpgroups, which exchange their partial sums through shared memory (an
 //            mbarrier, so the wait stays bounded); a second pass over the same registers
 //            scales by rstd * w and stores. Columns past n_norm_cols pass through.
+//   POINTWISE y = act(alpha * acc + bias[col]) (act: none or ReLU), cast to bf16, f16 or f32
+//            (section "Epilogue fusion in brief": bias, ReLU and cast, each element on its
+//            own); optional NVFP4 quantisation of bf16(y) with a static scale, the next
+//            layer's input.
 //   SWIGLU   accumulator columns come interleaved [g0, u0, g1, u1, ...] from the weight
 //            packing of section "Fusing gated SiLU (SwiGLU)", so each thread computes
 //            silu(g) * u on adjacent columns of its own row; optional NVFP4
@@ -44,7 +48,8 @@
 
 namespace nvfp4 {
 
-enum EpiKind { EPI_PLAIN = 0, EPI_RMSNORM = 1, EPI_SWIGLU = 2 };
+enum EpiKind { EPI_PLAIN = 0, EPI_RMSNORM = 1, EPI_SWIGLU = 2, EPI_POINTWISE = 3 };
+enum OutKind { OUT_BF16 = 0, OUT_F16 = 1, OUT_F32 = 2 };
 
 namespace gemm_cfg {
 constexpr int BM = 128;                 // output rows per CTA
@@ -222,12 +227,16 @@ struct GemmArgs {
   int head_dim;
   int n_norm_cols;
   float eps;
+  // pointwise
+  const float* bias;    // N floats, 16-byte aligned (or null)
+  int act;              // 0 none, 1 ReLU
+  int out_kind;         // OutKind of D
   // outputs
-  int write_d;          // bf16 output through tmD
-  uint8_t* q_codes;     // SwiGLU re-quantised output (or null)
+  int write_d;          // D through tmD (bf16, or out_kind for POINTWISE)
+  uint8_t* q_codes;     // NVFP4 quantised output (or null): SwiGLU, POINTWISE
   uint8_t* q_sf;
   const float* q_gscale;
-  int q_cols;           // Nh
+  int q_cols;           // its columns (Nh, or N)
   uint64_t wait_limit_ns;
 };
 
@@ -340,6 +349,72 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, i
       dst[0] = make_uint4(qc[0], qc[1], qc[2], qc[3]);
       dst[1] = make_uint4(qc[4], qc[5], qc[6], qc[7]);
       *reinterpret_cast<uint32_t*>(args.q_sf + sf_word_offset(row, oc0 >> 4, args.q_cols >> 4)) = sfw;
+    }
+    return true;
+  } else if constexpr (EPI == EPI_POINTWISE) {
+    // y = act(alpha * acc + bias[col]) in place of the accumulator bits
+    const float4* bp = reinterpret_cast<const float4*>(args.bias + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 b = args.bias != nullptr ? __ldg(bp + 8 * q + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float y = __fmaf_rn(alpha, __uint_as_float(v[q][4 * j4 + e]), bb[e]);
+          if (args.act == 1) y = fmaxf(y, 0.0f);
+          v[q][4 * j4 + e] = __float_as_uint(y);
+        }
+      }
+    }
+    if (args.write_d) {
+      if (args.out_kind == OUT_F32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          box_reuse_wait(lane);
+          stage_row_bf16(c.box, lane, v[q]);  // 32 words: 32 floats of the row
+          flush_box(c.tmD, c.box, lane, col0 + 32 * q, m0 + c.sub * 32);
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t p[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const uint32_t* src = v[2 * h + (j >> 4)];
+            const float lo = __uint_as_float(src[2 * (j & 15)]), hi = __uint_as_float(src[2 * (j & 15) + 1]);
+            p[j] = args.out_kind == OUT_F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+          }
+          box_reuse_wait(lane);
+          stage_row_bf16(c.box, lane, p);
+          flush_box(c.tmD, c.box, lane, col0 + 64 * h, m0 + c.sub * 32);
+        }
+      }
+    }
+    if (args.q_codes != nullptr) {
+      const int64_t row = m0 + row_in_tile;
+      uint4* dst = reinterpret_cast<uint4*>(args.q_codes + row * (args.q_cols >> 1) + (col0 >> 1));
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        uint32_t sfw = 0u;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {  // 32 values: two 16-blocks, 16 bytes of codes
+          uint32_t qc[4];
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            const int blk = 4 * w + 2 * k + hb;
+            const uint32_t* src = v[blk >> 1] + 16 * (blk & 1);
+            uint32_t p[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              p[j] = pack_bf16x2(__uint_as_float(src[2 * j]), __uint_as_float(src[2 * j + 1]));
+            sfw |= quant_block16_bf16(p, c.qG, c.qenc, qc[2 * hb], qc[2 * hb + 1]) << (8 * (2 * k + hb));
+          }
+          dst[2 * w + k] = make_uint4(qc[0], qc[1], qc[2], qc[3]);
+        }
+        *reinterpret_cast<uint32_t*>(args.q_sf + sf_word_offset(row, (col0 >> 4) + 4 * w, args.q_cols >> 4)) = sfw;
+      }
     }
     return true;
   } else {

@@ -30,9 +30,9 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sm_count = 0;
-  bool gemm_attr_set[3] = {false, false, false};
-  bool pair_attr_set[3] = {false, false, false};
-  int pair_clusters[3] = {0, 0, 0};
+  bool gemm_attr_set[4] = {false, false, false, false};
+  bool pair_attr_set[4] = {false, false, false, false};
+  int pair_clusters[4] = {0, 0, 0, 0};
   bool quant_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -113,9 +113,11 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   if (B.cols != K) return NVFP4_ERR_INVALID_ARG;
   if (M % BM || N % BN || K % BK) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (M > (1ll << 30) || N > (1ll << 30) || K > (1ll << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const int out_kind = EPI == nvfp4::EPI_POINTWISE ? args.out_kind : nvfp4::OUT_BF16;
+  const int esize = out_kind == nvfp4::OUT_F32 ? 4 : 2;
   if (D != nullptr) {
     if (ldd < n_out) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(D) || (ldd % 8) != 0) return NVFP4_ERR_MISALIGNED;
+    if (!aligned16(D) || (ldd * esize) % 16 != 0) return NVFP4_ERR_MISALIGNED;
   }
   int dev;
   DeviceInfo* info;
@@ -137,8 +139,12 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return NVFP4_ERR_CUDA;
   }
-  if (D != nullptr &&
-      !make_map_2d(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, n_out, M, ldd * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+  // D staged by 32 rows x 128 bytes and stored by TMA: 64 columns of bf16/f16 or 32 of f32
+  const CUtensorMapDataType d_type = out_kind == nvfp4::OUT_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                     : out_kind == nvfp4::OUT_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (D != nullptr && !make_map_2d(&tmD, d_type, D, n_out, M, ldd * esize, 128 / esize, 32,
+                                   CU_TENSOR_MAP_SWIZZLE_128B))
     return NVFP4_ERR_CUDA;
 
   args.sfa = static_cast<const uint8_t*>(A.sf);
@@ -328,6 +334,30 @@ NVFP4_API nvfp4_status gemm_nvfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D,
   if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
   nvfp4::GemmArgs args{};
   return run_gemm<nvfp4::EPI_PLAIN>(A, B, D, ldd, B.rows, args, stream);
+}
+
+NVFP4_API nvfp4_status gemm_nvfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* bias, int act,
+                                            int out_dtype, void* D, int64_t ldd, const nvfp4_tensor* Dq,
+                                            cudaStream_t stream) {
+  if (D == nullptr && Dq == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (act != NVFP4_ACT_NONE && act != NVFP4_ACT_RELU) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
+    return NVFP4_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return NVFP4_ERR_MISALIGNED;
+  nvfp4::GemmArgs args{};
+  args.bias = bias;
+  args.act = act;
+  args.out_kind = out_dtype;
+  if (Dq != nullptr) {
+    if (Dq->codes == nullptr || Dq->sf == nullptr || Dq->gscale == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (Dq->rows != A.rows || Dq->cols != B.rows) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(Dq->codes) || !aligned16(Dq->sf)) return NVFP4_ERR_MISALIGNED;
+    args.q_codes = static_cast<uint8_t*>(Dq->codes);
+    args.q_sf = static_cast<uint8_t*>(Dq->sf);
+    args.q_gscale = Dq->gscale;
+    args.q_cols = static_cast<int>(B.rows);
+  }
+  return run_gemm<nvfp4::EPI_POINTWISE>(A, B, D, ldd, B.rows, args, stream);
 }
 
 NVFP4_API nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,

@@ -308,21 +308,54 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
             word |= quant_block16_bf16(w, G, enc, cw[2 * blk], cw[2 * blk + 1]) << (8 * blk);
           }
           if (a.codes != nullptr) {
-            if (r < a.rows) {
-              uint4* dst = reinterpret_cast<uint4*>(a.codes + r * (a.cols >> 1) + g * 32);
-              dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-              dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            // 32 bytes of codes per row: staged in the row's first two chunks of the stage,
+            // then stored as whole 32-byte sectors, lanes 2k and 2k+1 taking the halves of
+            // one row, 16 rows per instruction
+            uint8_t* mine = smem + stage * STAGE_BYTES + rowoff;
+            *reinterpret_cast<uint4*>(mine + ((0 ^ sw) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            *reinterpret_cast<uint4*>(mine + ((1 ^ sw) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            __syncwarp();
+            const int i0 = i - lane;
+            const int hf = lane & 1;
+#pragma unroll
+            for (int rd = 0; rd < 2; ++rd) {
+              const int ii = i0 + 16 * rd + (lane >> 1);
+              const int sri = a.interleave ? ((ii & 1) ? R / 2 + (ii >> 1) : (ii >> 1)) : ii;
+              const int64_t rr = rs * R + ii;
+              if (rr < a.rows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(smem + stage * STAGE_BYTES + b * R * 128 + sri * 128 +
+                                                                  ((hf ^ (sri & 7)) << 4));
+                *reinterpret_cast<uint4*>(a.codes + rr * (a.cols >> 1) + g * 32 + hf * 16) = val;
+              }
             }
             *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(r, 4 * g, a.cols >> 4)) = word;
           }
-          if (a.y != nullptr && r < a.rows) {
-            uint4* dst = reinterpret_cast<uint4*>(a.y + r * a.ldy + g * 64);
+          if (a.y != nullptr) {
+            // The warp's 32 rows of y go back into its own rows of the stage (same swizzle),
+            // then leave as whole 128-byte lines: lanes 8k..8k+7 store the 8 chunks of one
+            // row, 4 rows per instruction.
+            __syncwarp();  // the code transposition above has read the stage rows
+            uint8_t* mine = smem + stage * STAGE_BYTES + rowoff;
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
               uint32_t o[8];
               dequant_block16_bf16(cw[2 * blk], cw[2 * blk + 1], (word >> (8 * blk)) & 0xFFu, G, o);
-              dst[2 * blk] = make_uint4(o[0], o[1], o[2], o[3]);
-              dst[2 * blk + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+              *reinterpret_cast<uint4*>(mine + (((2 * blk) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(mine + (((2 * blk + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            __syncwarp();
+            const int i0 = i - lane;  // the warp's first row of the box
+            const int ch = lane & 7;
+#pragma unroll
+            for (int rd = 0; rd < 8; ++rd) {
+              const int ii = i0 + 4 * rd + (lane >> 3);
+              const int sri = a.interleave ? ((ii & 1) ? R / 2 + (ii >> 1) : (ii >> 1)) : ii;
+              const int64_t rr = rs * R + ii;
+              if (rr < a.rows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(smem + stage * STAGE_BYTES + b * R * 128 + sri * 128 +
+                                                                  ((ch ^ (sri & 7)) << 4));
+                *reinterpret_cast<uint4*>(a.y + rr * a.ldy + g * 64 + ch * 8) = val;
+              }
             }
           }
         }

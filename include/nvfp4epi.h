@@ -133,6 +133,31 @@ nvfp4_status gemm_nvfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t l
                               cudaStream_t stream);
 
 /*
+ * Pointwise epilogue on the plain GEMM ("Serving sub-second Ideogram v4 without quality
+ * loss", section "Epilogue fusion in brief": bias, ReLU and cast, each output element on
+ * its own):
+ *   y[m,n] = act(fma(G_A * G_B, acc[m,n], bias[n]))   (float32; act: none or ReLU)
+ *   D = y cast to out_dtype (round to nearest even), and/or
+ *   Dq = NVFP4 of bf16(y) with the static scale *Dq->gscale (as nvfp4_quantize with
+ *        compute_amax = 0 would give for bf16(y)): the next layer's input.
+ *   bias: N float32, 16-byte aligned, or NULL (no bias).
+ *   act: NVFP4_ACT_NONE or NVFP4_ACT_RELU.
+ *   out_dtype: NVFP4_OUT_BF16, NVFP4_OUT_F16 or NVFP4_OUT_F32; D is M x N of that type with
+ *              leading dimension ldd elements (ldd * element size a multiple of 16 bytes),
+ *              or NULL.
+ *   Dq: M x N NVFP4 (codes 16-byte aligned, scales in the tensor-core layout), or NULL.
+ * Shape rules as gemm_nvfp4_plain; D and Dq may not both be NULL.
+ */
+#define NVFP4_ACT_NONE 0
+#define NVFP4_ACT_RELU 1
+#define NVFP4_OUT_BF16 0
+#define NVFP4_OUT_F16 1
+#define NVFP4_OUT_F32 2
+nvfp4_status gemm_nvfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* bias, int act,
+                                  int out_dtype, void* D, int64_t ldd, const nvfp4_tensor* Dq,
+                                  cudaStream_t stream);
+
+/*
  * As gemm_nvfp4_plain, then per row and per head of head_dim adjacent columns among the
  * first n_norm_cols: y = x * rsqrt(mean(x^2) + eps) * w[col] (x = G_A G_B acc, float32);
  * columns >= n_norm_cols pass through (the V block of a QKV projection).

@@ -307,6 +307,21 @@ def rmsnorm_heads(x, w, head_dim: int, n_norm_cols: int, eps: float) -> np.ndarr
     return y
 
 
+def pointwise(c, bias=None, relu: bool = False) -> np.ndarray:
+    """Pointwise epilogue of page "Serving sub-second Ideogram v4 without quality loss",
+    section "Epilogue fusion in brief" (bias, ReLU, cast): y = act(c + bias[n]) for an
+    alpha-scaled accumulator c. The sum is rounded once to float32 (the GPU forms
+    alpha * acc + bias with one fused multiply-add); returned as float64 holding float32
+    values, ready for the cast (bf16_round, or numpy's float16/float32)."""
+    y = np.asarray(c, np.float64)
+    if bias is not None:
+        y = y + np.asarray(bias, np.float64)[None, :]
+    y = y.astype(F32).astype(np.float64)
+    if relu:
+        y = np.maximum(y, 0.0)
+    return y
+
+
 def silu(x) -> np.ndarray:
     x = np.asarray(x, np.float64)
     with np.errstate(over="ignore"):
@@ -376,6 +391,10 @@ def problem_plain(a_bf16, b_bf16, rows=None, b_quant=None) -> np.ndarray:
 def problem_rmsnorm(a_bf16, b_bf16, w, head_dim, n_norm_cols, eps, rows=None, b_quant=None) -> np.ndarray:
     c = problem_gemm(a_bf16, b_bf16, rows, b_quant)
     return bf16_round(rmsnorm_heads(c, w, head_dim, n_norm_cols, eps))
+
+
+def problem_pointwise(a_bf16, b_bf16, bias=None, relu=False, rows=None, b_quant=None) -> np.ndarray:
+    return pointwise(problem_gemm(a_bf16, b_bf16, rows, b_quant), bias, relu)
 
 
 def problem_swiglu(a_bf16, b_gate_up_bf16, rows=None, b_quant=None) -> np.ndarray:

@@ -126,3 +126,18 @@ def test_problem_pipeline_small(M, N, K):
     ref = a.double().numpy() @ b.double().numpy().T
     rel = np.linalg.norm(c - ref) / np.linalg.norm(ref)
     assert rel < 0.3
+
+
+def test_pointwise_matches_torch_float32_bias_add_and_relu():
+    rng = np.random.default_rng(4)
+    c = rng.standard_normal((64, 96)).astype(np.float32).astype(np.float64)  # float32-valued
+    bias = (rng.standard_normal(96) * 3).astype(np.float32)
+    got = o.pointwise(c, bias, relu=True)
+    ref = torch.relu(torch.from_numpy(c.astype(np.float32)) + torch.from_numpy(bias)).double().numpy()
+    assert np.array_equal(got, ref)
+    # no bias, no activation: the float32 rounding of c only
+    c2 = rng.standard_normal((8, 32))
+    assert np.array_equal(o.pointwise(c2), c2.astype(np.float32).astype(np.float64))
+    # ReLU zeroes exactly the negative sums
+    y = o.pointwise(c, bias)
+    assert np.array_equal(o.pointwise(c, bias, relu=True) == 0, y <= 0)
