@@ -1,0 +1,45 @@
+"""TPLayer on one GPU (no process group: world size 1) computes exactly what the
+unsharded kernels do: the shard packing with the whole weights' scales, the QKV shard's
+normalised-column count and the f32 partial-sum path of the row-parallel down GEMM."""
+import numpy as np
+import pytest
+import torch
+
+import epilogues_nvfp4_quantize_b200 as ep
+from epilogues_nvfp4_quantize_b200.parallel import TPLayer
+import workloads as wk
+from gpu_util import device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M", [256, 384])
+def test_tp_layer_world1_equals_the_unsharded_kernels(M):
+    dev = device()
+    heads, hd, K, nh = 4, 128, 512, 512
+    x = wk.activations(M, K, 1, seed=M).to(dev)
+    wq = wk.weights(3 * heads * hd, K, 1 / np.sqrt(K), seed=1).to(dev)
+    wu = wk.weights(2 * nh, K, 1 / np.sqrt(K), seed=2).to(dev)
+    wd = wk.weights(K, nh, 1 / np.sqrt(nh), seed=3).to(dev)
+    wn_q = torch.from_numpy(wk.norm_weight(hd, 0, 3)).to(dev)
+    wn_k = torch.from_numpy(wk.norm_weight(hd, 0, 5)).to(dev)
+    T = ep.NVFP4Tensor
+    xq = ep.nvfp4_quantize(x, T.empty(M, K, dev))
+    G_h = 0.01
+    layer = TPLayer(wq, wu, wd, wn_q, wn_k, heads, hd, G_h)
+    qkv, out = layer.step(xq)
+
+    Wq = ep.nvfp4_quantize(wq, T.empty(wq.shape[0], K, dev))
+    Wu = ep.nvfp4_quantize(wu, T.empty(wu.shape[0], K, dev), interleave=True)
+    Wd = ep.nvfp4_quantize(wd, T.empty(K, nh, dev))
+    w_norm = torch.cat([wn_q.repeat(heads), wn_k.repeat(heads)]).float().contiguous()
+    qkv_ref = torch.empty_like(qkv)
+    ep.gemm_nvfp4_rmsnorm(xq, Wq, w_norm, hd, 2 * heads * hd, 1e-6, qkv_ref)
+    h = T.empty(M, nh, dev)
+    h.gscale.fill_(G_h)
+    ep.gemm_nvfp4_swiglu(xq, Wu, None, h)
+    out_ref = torch.empty(M, K, dtype=torch.float32, device=dev)
+    ep.gemm_nvfp4_pointwise(h, Wd, out_ref)
+    assert torch.equal(qkv, qkv_ref)
+    assert torch.equal(out, out_ref)
+    assert ep.read_device_status() == 0
