@@ -405,3 +405,84 @@ def problem_swiglu(a_bf16, b_gate_up_bf16, rows=None, b_quant=None) -> np.ndarra
 def requantize(out_bf16_values, G):
     """Static-scale NVFP4 quantisation of bf16-valued outputs (blocks along N)."""
     return quantize(np.asarray(out_bf16_values, np.float64).astype(F32), G)
+
+
+# ----------------------------------------------------------------------------------
+# MXFP4 with a block-local transform (page "KroQuant: efficient post-training
+# quantization for diffusion transformers via Kronecker-product structure": activations
+# split into independent blocks of 32, each with an invertible Kronecker-structured
+# transform; MXFP4 format). The pages' transforms are learned; this build uses a fixed
+# one, the 32-point Walsh-Hadamard matrix H_2 (x) H_2 (x) H_2 (x) H_2 (x) H_2.
+# MXFP4 per the OCP Microscaling format: E2M1 elements, one E8M0 (power-of-two) scale
+# per 32 elements, no per-tensor scale.
+# ----------------------------------------------------------------------------------
+
+MX_BLOCK = 32
+
+
+def e8m0_decode(codes) -> np.ndarray:
+    """E8M0 scale code e -> 2^(e - 127) (float64; code 255 is NaN and never produced)."""
+    e = np.asarray(codes, dtype=np.int64)
+    return np.ldexp(1.0, e - 127)
+
+
+def mx_quantize(x):
+    """Quantise (rows, cols) float32 to MXFP4, blocks of 32 along cols. Per block: the
+    shared exponent is floor(log2(amax)) - 2 (2 = the exponent of E2M1's largest value,
+    6 = 1.5 * 2^2), clamped to [-127, 127]; the scale is X = 2^that; elements are
+    E2M1_rn_satfinite(x / X) (x / X is exact: X is a power of two). An all-zero block gets
+    code 0 and zero elements. Returns (codes (rows, cols) uint8, e8m0 (rows, cols/32))."""
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    xb = x.reshape(rows, cols // MX_BLOCK, MX_BLOCK).astype(np.float64)
+    amax = np.abs(xb).max(axis=2)
+    _, p = np.frexp(amax)                      # amax = m * 2^p, 0.5 <= m < 1
+    shared = np.clip(p - 1 - 2, -127, 127)     # floor(log2 amax) - 2
+    e = np.where(amax > 0, shared + 127, 0).astype(np.uint8)
+    X = np.ldexp(1.0, shared)[:, :, None]
+    q = e2m1_encode((xb / X).astype(F32).reshape(rows, cols))
+    q = np.where(np.repeat(amax > 0, MX_BLOCK, axis=1), q, 0).astype(np.uint8)
+    return q, e
+
+
+def mx_dequantize(codes, e8m0) -> np.ndarray:
+    """dec(q) * 2^(e - 127) in float64, (rows, cols)."""
+    codes = np.asarray(codes)
+    rows, cols = codes.shape
+    vals = _E2M1_TABLE[codes & 0xF].reshape(rows, cols // MX_BLOCK, MX_BLOCK)
+    vals *= e8m0_decode(e8m0)[:, :, None]
+    return vals.reshape(rows, cols)
+
+
+def hadamard32(x) -> np.ndarray:
+    """x @ H32 per block of 32 along cols, H32 the unnormalised Sylvester-Hadamard matrix
+    (entries +-1), computed in float32 by the fast Walsh-Hadamard transform: five stages,
+    stage h in (1, 2, 4, 8, 16) maps each pair (j, j + h), j with bit h clear, to
+    (a + b, a - b). H32 H32^T = 32 I, so (x H)(w H)^T = 32 x w^T."""
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    y = x.reshape(rows, cols // MX_BLOCK, MX_BLOCK).copy()
+    h = 1
+    while h < MX_BLOCK:
+        y = y.reshape(rows, cols // MX_BLOCK, MX_BLOCK // (2 * h), 2, h)
+        a, b = y[:, :, :, 0, :].copy(), y[:, :, :, 1, :].copy()
+        y[:, :, :, 0, :] = a + b
+        y[:, :, :, 1, :] = a - b
+        h *= 2
+    return y.reshape(rows, cols)
+
+
+def mx_sf_bytes(rows: int, cols: int) -> int:
+    """Size of an MXFP4 scale buffer: the tensor-core scale layout with 32-blocks (a
+    512-byte unit holds 128 rows x 4 blocks, i.e. 128 K values)."""
+    return sf_bytes(rows, cols // 2)
+
+
+def mx_pack_scales(e8m0, cols: int) -> np.ndarray:
+    """(rows, cols/32) E8M0 codes -> flat layout buffer: the same unit layout as
+    pack_scales, counting blocks of 32 (so it is pack_scales at half the columns)."""
+    return pack_scales(e8m0, cols // 2)
+
+
+def mx_unpack_scales(buf, rows: int, cols: int) -> np.ndarray:
+    return unpack_scales(buf, rows, cols // 2)

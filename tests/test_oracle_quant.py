@@ -166,3 +166,51 @@ def test_fake_quantize_is_odd_and_close_to_the_exact_dequantisation():
 def test_fake_quantize_of_zero_is_zero():
     y, G = o.fake_quantize(np.zeros((128, 64), np.float32))
     assert G == 0 and not y.any()
+
+
+# ---- MXFP4 and the block Hadamard transform ---------------------------------------
+
+def test_hadamard32_matches_scipy_and_is_its_own_inverse_up_to_32():
+    import scipy.linalg
+    H = scipy.linalg.hadamard(32).astype(np.float64)  # Sylvester construction, a library routine
+    x = _rand(16, 128, seed=12)
+    y = o.hadamard32(x)
+    ref = (x.astype(np.float64).reshape(16, 4, 32) @ H).reshape(16, 128)
+    assert np.allclose(y, ref, rtol=1e-6, atol=1e-5)
+    xi = np.random.default_rng(2).integers(-8, 8, size=(8, 64)).astype(np.float32)  # exact in fp32
+    assert np.array_equal(o.hadamard32(o.hadamard32(xi)), 32 * xi)
+    assert np.array_equal((xi.reshape(8, 2, 32).astype(np.float64) @ H).reshape(8, 64), o.hadamard32(xi))
+
+
+def test_mx_quantize_scale_rule_and_bounds():
+    x = _rand(64, 256, seed=13, outliers=2)
+    q, e = o.mx_quantize(x)
+    xb = x.reshape(64, 8, 32)
+    amax = np.abs(xb).max(axis=2)
+    X = o.e8m0_decode(e)
+    # the shared exponent puts amax / X in [4, 8): one power of two below E2M1's top level
+    assert np.all((amax / X >= 4) & (amax / X < 8))
+    deq = o.mx_dequantize(q, e)
+    # error within half the widest level step (2) of the block, or the saturation of
+    # values above 6 X
+    err = np.abs(deq - x).reshape(64, 8, 32)
+    bound = np.maximum(1.0 * X, amax - 6 * X)[:, :, None]
+    assert np.all(err <= bound + 1e-12)
+    # exact on representable blocks: levels times a power of two, top level present
+    lv = o.e2m1_decode(np.arange(16))
+    qq = np.random.default_rng(1).integers(0, 16, size=(4, 64))
+    qq[:, ::32] = 7
+    xr = (lv[qq] * 2.0 ** -5).astype(np.float32)
+    q2, e2 = o.mx_quantize(xr)
+    assert np.array_equal(o.mx_dequantize(q2, e2), xr.astype(np.float64))
+    assert np.all(e2 == 127 - 5)
+
+
+def test_mx_zero_block_and_layout_roundtrip():
+    x = _rand(128, 256, seed=14)
+    x[3, 32:64] = 0
+    q, e = o.mx_quantize(x)
+    assert e[3, 1] == 0 and not q[3, 32:64].any()
+    buf = o.mx_pack_scales(e, 256)
+    assert buf.size == o.mx_sf_bytes(128, 256) == 128 * 8
+    assert np.array_equal(o.mx_unpack_scales(buf, 128, 256), e)
