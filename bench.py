@@ -379,6 +379,27 @@ def run_cuda(args):
         result["pointwise"] = pw
         del d32, dq
 
+    # ---- MXFP4 with the block Hadamard transform: same GEMM shapes, E8M0 scales per 32
+    if not args.no_unfused:
+        T = ep.NVFP4Tensor
+        xm = ep.mxfp4_quantize(layer.x, T.empty_mx(M, K_IN, dev), hadamard=True)
+        w_up_bf16 = torch.randn(N_UP, K_IN, device=dev, dtype=torch.bfloat16) * (1.0 / K_IN ** 0.5)
+        wm = ep.mxfp4_quantize(w_up_bf16, T.empty_mx(N_UP, K_IN, dev), hadamard=True)
+        c_mx = torch.empty(M, N_UP, dtype=torch.bfloat16, device=dev)
+        c_nv = torch.empty(M, N_UP, dtype=torch.bfloat16, device=dev)
+        barrier()
+        t_mx = time_loop(lambda: ep.gemm_mxfp4_plain(xm, wm, c_mx), args.cmp_steps, 3, torch)
+        t_nv = time_loop(lambda: ep.gemm_nvfp4_plain(layer.xq, layer.Wup_logical, c_nv), args.cmp_steps, 3, torch)
+        t_q = time_loop(lambda: ep.mxfp4_quantize(layer.x, xm, hadamard=True), args.cmp_steps, 3, torch)
+        result["mxfp4"] = {
+            "shape": f"M={M} K={K_IN} N={N_UP} (FFN-up, bf16 out, no epilogue op)",
+            "gemm_us": round(t_mx * 1e3, 1), "gemm_tflops": round(flops["up"] / (t_mx * 1e-3) / 1e12, 1),
+            "nvfp4_same_shape_us": round(t_nv * 1e3, 1),
+            "quantize_hadamard_us": round(t_q * 1e3, 1),
+            "quantize_gbs": round(layer.x.numel() * (2 + 0.5 + 1 / 32) / (t_q * 1e-3) / 1e9, 1),
+        }
+        del xm, wm, c_mx, c_nv, w_up_bf16
+
     # ---- fake quantisation (quantization-aware distillation forward), HBM-bound
     if not args.no_unfused:
         y_fq = torch.empty_like(layer.x)

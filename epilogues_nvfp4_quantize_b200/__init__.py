@@ -8,11 +8,14 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     FakeQuantizeSTE,
     NVFP4Tensor,
+    gemm_mxfp4_plain,
+    gemm_mxfp4_pointwise,
     gemm_nvfp4_plain,
     gemm_nvfp4_pointwise,
     gemm_nvfp4_rmsnorm,
     gemm_nvfp4_swiglu,
     launch_count,
+    mxfp4_quantize,
     load,
     nvfp4_fake_quantize,
     nvfp4_quantize,

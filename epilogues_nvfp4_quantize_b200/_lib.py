@@ -25,6 +25,7 @@ EXPORTS = (
     "rmsnorm_heads_bf16", "swiglu_bf16", "nvfp4_status_string",
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
     "nvfp4_quantize_noalloc", "nvfp4_fake_quantize", "gemm_nvfp4_pointwise",
+    "mxfp4_sf_bytes", "mxfp4_quantize", "gemm_mxfp4_pointwise", "gemm_mxfp4_plain",
 )
 
 
@@ -61,6 +62,10 @@ def load() -> ctypes.CDLL:
         "nvfp4_quantize_noalloc": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
         "nvfp4_fake_quantize": (i32, [vp, i64, i64, i64, i32, vp, vp, i64, vp, vp]),
         "gemm_nvfp4_pointwise": (i32, [_Tensor, _Tensor, vp, i32, i32, vp, i64, ctypes.POINTER(_Tensor), vp]),
+        "mxfp4_sf_bytes": (i64, [i64, i64]),
+        "mxfp4_quantize": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
+        "gemm_mxfp4_pointwise": (i32, [_Tensor, _Tensor, vp, i32, i32, vp, i64, vp]),
+        "gemm_mxfp4_plain": (i32, [_Tensor, _Tensor, vp, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -96,6 +101,13 @@ class NVFP4Tensor:
     def empty(cls, rows: int, cols: int, device="cuda") -> "NVFP4Tensor":
         return cls(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
                    torch.empty((sf_bytes(rows, cols),), dtype=torch.uint8, device=device),
+                   torch.empty((1,), dtype=torch.float32, device=device), rows, cols)
+
+    @classmethod
+    def empty_mx(cls, rows: int, cols: int, device="cuda") -> "NVFP4Tensor":
+        """Buffers of an MXFP4 tensor (E8M0 scales per 32 values; see mxfp4_quantize)."""
+        return cls(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+                   torch.empty((int(load().mxfp4_sf_bytes(rows, cols)),), dtype=torch.uint8, device=device),
                    torch.empty((1,), dtype=torch.float32, device=device), rows, cols)
 
     def c(self) -> _Tensor:
@@ -179,6 +191,36 @@ def gemm_nvfp4_pointwise(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tenso
     _check(load().gemm_nvfp4_pointwise(A.c(), B.c(), _ptr(bias), ACT_RELU if relu else ACT_NONE, kind, p, ld, dq,
                                        _stream(stream)), "gemm_nvfp4_pointwise")
     return D, Dq
+
+
+MXFP4_HADAMARD32 = 2
+
+
+def mxfp4_quantize(x: torch.Tensor, out: NVFP4Tensor, hadamard: bool = False, stream=None) -> NVFP4Tensor:
+    """MXFP4-quantise a bf16 2-D CUDA tensor (optionally after the 32-point block Hadamard
+    transform) into `out` (from NVFP4Tensor.empty_mx); see mxfp4_quantize in the header."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
+    _check(load().mxfp4_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0),
+                                 MXFP4_HADAMARD32 if hadamard else 0, out.c(), _stream(stream)), "mxfp4_quantize")
+    return out
+
+
+def gemm_mxfp4_pointwise(A: NVFP4Tensor, B: NVFP4Tensor, D: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                         relu: bool = False, stream=None) -> torch.Tensor:
+    if bias is not None and (bias.dtype != torch.float32 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous float32 tensor")
+    if D.dtype not in _OUT_KIND or D.dim() != 2 or D.stride(1) != 1:
+        raise ValueError("D must be a 2-D bf16, f16 or f32 tensor with unit column stride")
+    _check(load().gemm_mxfp4_pointwise(A.c(), B.c(), _ptr(bias), ACT_RELU if relu else ACT_NONE, _OUT_KIND[D.dtype],
+                                       D.data_ptr(), D.stride(0), _stream(stream)), "gemm_mxfp4_pointwise")
+    return D
+
+
+def gemm_mxfp4_plain(A: NVFP4Tensor, B: NVFP4Tensor, D: torch.Tensor, stream=None) -> torch.Tensor:
+    p, ld = _out2d(D)
+    _check(load().gemm_mxfp4_plain(A.c(), B.c(), p, ld, _stream(stream)), "gemm_mxfp4_plain")
+    return D
 
 
 def rmsnorm_heads_bf16(x: torch.Tensor, w: torch.Tensor, head_dim: int, n_norm_cols: int, eps: float,

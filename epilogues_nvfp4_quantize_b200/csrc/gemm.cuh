@@ -81,13 +81,21 @@ __host__ __device__ constexpr uint32_t sf_slot(uint32_t s) { return SF_SLOT0 + S
 static_assert(ACC_COL1 + 256 <= SF_SLOT0 && ACC_COL1 >= 128 && sf_slot(2) <= TMEM_COLS, "TMEM plan");
 }  // namespace gemm_cfg
 
+// Block-scale format: NVFP4 (E4M3 scale per 16 values) or MXFP4 (E8M0 scale per 32). A
+// 512-byte scale unit holds 128 rows x 4 scales, i.e. 64 (NVFP4) or 128 (MXFP4) K values.
+template <bool MX>
+struct ScaleFmt {
+  static constexpr int K_PER_UNIT = MX ? 128 : 64;
+  static constexpr int UNITS = gemm_cfg::BK / K_PER_UNIT;  // units per K step per 128 rows: 4 or 2
+};
+
 // Shared-memory plan of a kernel with S stages of B_ROWS rows of B per CTA.
-template <int S, int B_ROWS>
+template <int S, int B_ROWS, bool MX = false>
 struct SmemPlan {
   static constexpr int A_BYTES = gemm_cfg::BM * gemm_cfg::BK_BYTES;                 // 16 KB
   static constexpr int B_BYTES = B_ROWS * gemm_cfg::BK_BYTES;                       // 16 or 32 KB
-  static constexpr int SFA_BYTES = (gemm_cfg::BK / 64) * gemm_cfg::SF_UNIT;          // 2 KB
-  static constexpr int SFB_BYTES = 2 * (gemm_cfg::BK / 64) * gemm_cfg::SF_UNIT;      // 4 KB (256 rows)
+  static constexpr int SFA_BYTES = ScaleFmt<MX>::UNITS * gemm_cfg::SF_UNIT;         // 2 KB (1 KB MXFP4)
+  static constexpr int SFB_BYTES = 2 * ScaleFmt<MX>::UNITS * gemm_cfg::SF_UNIT;     // 4 KB (2 KB MXFP4), 256 rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int OFF_EPI = S * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
@@ -98,8 +106,12 @@ struct SmemPlan {
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
-using PlanSingle = SmemPlan<3, 256>;
-using PlanPair = SmemPlan<5, 128>;
+template <bool MX>
+using PlanSingleT = SmemPlan<3, 256, MX>;
+template <bool MX>
+using PlanPairT = SmemPlan<5, 128, MX>;
+using PlanSingle = PlanSingleT<false>;
+using PlanPair = PlanPairT<false>;
 
 // Barriers past the stage ring (full[S], empty[S]), at empty + S + index.
 namespace bar_idx {
@@ -147,12 +159,13 @@ __device__ __forceinline__ uint32_t ksteps_of(int num_tiles, int K, int first, i
 // Scale-copy warp `cw` (one elected lane). For K step g in stage `stage`: once the stage's
 // scale units have landed (they have their own barrier, so the copies overlap the arrival
 // of the larger code tiles) and the MMAs of step g - 2 have finished reading scale slot g % 2, copy its
-// share of the step's 12 scale units (unit i goes to warp i % COPY_WARPS) into that slot and
-// commit to sf_full[g % 2]. Slot layout: SFA of MMA q at columns 4q, SFB rows 0-127 of MMA q
-// at 16 + 8q, rows 128-255 at 16 + 8q + 4. In a CTA pair the leader copies for both CTAs and
+// share of the step's scale units (12 for NVFP4, 6 for MXFP4; unit i goes to warp
+// i % COPY_WARPS) into that slot and commit to sf_full[g % 2]. Slot layout: SFA unit q at
+// columns 4q, SFB rows 0-127 of unit q at 16 + 8q, rows 128-255 at 16 + 8q + 4. An NVFP4
+// unit serves one K = 64 MMA; an MXFP4 unit two (bytes 0-1 and 2-3 of each word). In a CTA pair the leader copies for both CTAs and
 // the commits go to the leader's barriers only. Returns false if a bounded wait gave up
 // (after waiting, bounded, for its own copies).
-template <bool PAIR, int STAGES, int STAGE_BYTES, int SF_OFF, int SFB_HALF>
+template <bool PAIR, bool MX, int STAGES, int STAGE_BYTES, int SF_OFF, int SFB_HALF>
 __device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* bars, uint32_t tmem,
                                                 int cw, uint32_t nsteps, volatile int* abort_flag, uint64_t limit,
                                                 int where) {
@@ -171,11 +184,12 @@ __device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* bars, u
       break;
     }
     tc_fence_after();
+    constexpr int U = ScaleFmt<MX>::UNITS;
     const uint32_t sfa = smem_u32(smem + stage * STAGE_BYTES) + SF_OFF;
-    const uint32_t sfb = sfa + (BK / 64) * SF_UNIT;
+    const uint32_t sfb = sfa + U * SF_UNIT;
     const uint32_t slot = tmem + sf_slot(s);
 #pragma unroll
-    for (int i = 0; i < 3 * (BK / 64); ++i) {
+    for (int i = 0; i < 3 * U; ++i) {
       if (i % COPY_WARPS != cw) continue;
       const int q = i / 3, r = i % 3;
       const uint32_t dst = r == 0 ? slot + 4 * q : slot + SFB_OFF + 8 * q + 4 * (r - 1);
@@ -509,12 +523,13 @@ __device__ __forceinline__ EpiCtx make_epi_ctx(const GemmArgs& args, const CUten
 // =====================================================================================
 // One CTA per 128 x 256 tile (used when M % 256 == 128)
 // =====================================================================================
-template <int EPI>
+template <int EPI, bool MX = false>
 __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
   using namespace gemm_cfg;
-  using P = PlanSingle;
+  using P = PlanSingleT<MX>;
+  constexpr int U = ScaleFmt<MX>::UNITS;
   constexpr int STAGES = 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -567,7 +582,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   const uint32_t tmem = *tmem_holder;
 
   const int ktiles = args.K / BK;
-  const int64_t kunits = args.K / 64;  // scale units per 128-row group along K
+  const int64_t kunits = args.K / ScaleFmt<MX>::K_PER_UNIT;  // scale units per 128-row group along K
 
   if (warp == EPI_WARPS) {
     // ------------------------------------------------------------------ producer
@@ -588,7 +603,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           // scales first, on their own barrier, then the code tiles
           uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
           mbar_arrive_expect_tx(sfl, P::SFA_BYTES + P::SFB_BYTES);
-          const int64_t ka = static_cast<int64_t>(kt) * (BK / 64);
+          const int64_t ka = static_cast<int64_t>(kt) * U;
           uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
           bulk_load(ssf, args.sfa + (tm * kunits + ka) * SF_UNIT, P::SFA_BYTES, sfl);
           bulk_load(ssf + P::SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT, P::SFB_BYTES / 2, sfl);
@@ -629,7 +644,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else if (warp == EPI_WARPS + 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_nvfp4(BM, BN);
+      const uint32_t idesc = MX ? idesc_mxfp4(BM, BN, 0) : idesc_nvfp4(BM, BN);
       int stage = 0;
       uint32_t phase = 0, j = 0, g = 0;
       bool ok = true;
@@ -656,8 +671,10 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
 #pragma unroll
           for (int kb = 0; kb < BK / 64; ++kb) {
             // +32 bytes along K per 64 FP4 values: +2 in the descriptor's address field
-            tc_mma_nvfp4(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, slot + 4 * kb, slot + SFB_OFF + 8 * kb,
-                         (kt > 0 || kb > 0) ? 1u : 0u);
+            const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
+            const uint32_t id = MX ? (idesc | ((2u * (kb & 1)) << 29) | ((2u * (kb & 1)) << 4)) : idesc;
+            tc_mma_nvfp4<MX>(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, id, slot + 4 * u, slot + SFB_OFF + 8 * u,
+                             (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           tc_commit(&xbars[bar_idx::SF_EMPTY + sl]);
@@ -677,7 +694,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else if (warp >= COPY_WARP0) {
     // ------------------------------------------------------------------ scale copies
     if (lane == 0) {
-      (void)scale_copy_loop<false, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+      (void)scale_copy_loop<false, MX, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
           smem, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
           abort_flag, limit, 14);
     }
@@ -715,13 +732,14 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
 // A CTA pair per 256 x 256 tile (used when M % 256 == 0). Cluster of 2 CTAs; CTA rank r
 // owns output rows [m0 + 128 r, m0 + 128 r + 128) and stages B rows [n0 + 128 r, +128).
 // =====================================================================================
-template <int EPI>
+template <int EPI, bool MX = false>
 __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                            const __grid_constant__ CUtensorMap tmD, const GemmArgs args) {
   using namespace gemm_cfg;
-  using P = PlanPair;
+  using P = PlanPairT<MX>;
+  constexpr int U = ScaleFmt<MX>::UNITS;
   constexpr int STAGES = 5;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -782,7 +800,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   const uint32_t tmem = *tmem_holder;
 
   const int ktiles = args.K / BK;
-  const int kunits = args.K / 64;
+  const int kunits = args.K / ScaleFmt<MX>::K_PER_UNIT;
 
   if (warp == EPI_WARPS) {
     // ------------------------------------------------------------------ producer (both CTAs)
@@ -811,10 +829,10 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           if (leader) mbar_arrive_expect_tx(sfl, 2 * (P::SFA_BYTES + P::SFB_BYTES));
           // scale units: 512 bytes = 2 rows of the 256-byte-wide scale tensor map
           uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
-          tma_load_2d_pair(ssf, &tmSFA, bar_sf, 0, 2 * (sfa_group * kunits + 4 * kt));
-          tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar_sf, 0, 2 * ((2 * tn) * kunits + 4 * kt));
+          tma_load_2d_pair(ssf, &tmSFA, bar_sf, 0, 2 * (sfa_group * kunits + U * kt));
+          tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar_sf, 0, 2 * ((2 * tn) * kunits + U * kt));
           tma_load_2d_pair(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, &tmSFB, bar_sf, 0,
-                           2 * ((2 * tn + 1) * kunits + 4 * kt));
+                           2 * ((2 * tn + 1) * kunits + U * kt));
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (P::A_BYTES + P::B_BYTES));
           tma_load_2d_pair(sb, &tmA, bar, kt * BK_BYTES, a_row);
           tma_load_2d_pair(sb + P::A_BYTES, &tmB, bar, kt * BK_BYTES, b_row);
@@ -848,7 +866,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else if (warp == EPI_WARPS + 1) {
     // ------------------------------------------------------------------ MMA issuer (leader only)
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_nvfp4(2 * BM, BN);
+      const uint32_t idesc = MX ? idesc_mxfp4(2 * BM, BN, 0) : idesc_nvfp4(2 * BM, BN);
       int stage = 0;
       uint32_t phase = 0, j = 0, g = 0;
       bool ok = true;
@@ -874,8 +892,10 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           const uint64_t bdesc = smem_desc_sw128(b_addr);
 #pragma unroll
           for (int kb = 0; kb < BK / 64; ++kb) {
-            tc_mma_nvfp4_pair(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, idesc, slot + 4 * kb, slot + SFB_OFF + 8 * kb,
-                              (kt > 0 || kb > 0) ? 1u : 0u);
+            const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
+            const uint32_t id = MX ? (idesc | ((2u * (kb & 1)) << 29) | ((2u * (kb & 1)) << 4)) : idesc;
+            tc_mma_nvfp4_pair<MX>(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, id, slot + 4 * u, slot + SFB_OFF + 8 * u,
+                                  (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
           tc_commit_pair(&xbars[bar_idx::SF_EMPTY + sl], 0x1);
@@ -895,7 +915,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else if (warp >= COPY_WARP0) {
     // ------------------------------------------------------------------ scale copies (leader only)
     if (leader && lane == 0) {
-      (void)scale_copy_loop<true, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+      (void)scale_copy_loop<true, MX, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
           smem, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
           abort_flag, limit, 31);
     }

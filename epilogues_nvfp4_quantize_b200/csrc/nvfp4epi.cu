@@ -30,9 +30,10 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sm_count = 0;
-  bool gemm_attr_set[4] = {false, false, false, false};
-  bool pair_attr_set[4] = {false, false, false, false};
-  int pair_clusters[4] = {0, 0, 0, 0};
+  // per kernel instance: index epilogue kind + 4 * (MXFP4 scales)
+  bool gemm_attr_set[8] = {};
+  bool pair_attr_set[8] = {};
+  int pair_clusters[8] = {};
   bool quant_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -102,7 +103,7 @@ nvfp4_status check_operand(const nvfp4_tensor& t) {
 
 // Common checks and launch of the GEMM kernels: the CTA-pair kernel when M % 256 == 0,
 // the single-CTA kernel otherwise.
-template <int EPI>
+template <int EPI, bool MX = false>
 nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int64_t ldd, int64_t n_out,
                       nvfp4::GemmArgs args, cudaStream_t stream) {
   using namespace nvfp4::gemm_cfg;
@@ -133,9 +134,12 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
     return NVFP4_ERR_CUDA;
   if (pair) {
     // the block scales seen as rows of 256 bytes; one 128-row x 256-K group = 8 rows
-    if (!make_map_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.sf, 256, M * (K / 16) / 256, 256, 256, 8,
+    // (NVFP4, a scale per 16 values) or 4 rows (MXFP4, a scale per 32)
+    const int64_t per_scale = MX ? 32 : 16;
+    const uint32_t box_rows = MX ? 4 : 8;
+    if (!make_map_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.sf, 256, M * (K / per_scale) / 256, 256, 256, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B.sf, 256, N * (K / 16) / 256, 256, 256, 8,
+        !make_map_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, B.sf, 256, N * (K / per_scale) / 256, 256, 256, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return NVFP4_ERR_CUDA;
   }
@@ -163,14 +167,14 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   args.wait_limit_ns = kWaitLimitNs;
 
   if (!pair) {
-    using P = nvfp4::PlanSingle;
-    auto kern = nvfp4::gemm_nvfp4_kernel<EPI>;
+    using P = nvfp4::PlanSingleT<MX>;
+    auto kern = nvfp4::gemm_nvfp4_kernel<EPI, MX>;
     {
       std::lock_guard<std::mutex> lock(g_mutex);
-      if (!info->gemm_attr_set[EPI]) {
+      if (!info->gemm_attr_set[EPI + 4 * MX]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
           return NVFP4_ERR_CUDA;
-        info->gemm_attr_set[EPI] = true;
+        info->gemm_attr_set[EPI + 4 * MX] = true;
       }
     }
     const int grid = args.num_tiles < info->sm_count ? args.num_tiles : info->sm_count;
@@ -179,8 +183,8 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
     return launch_status();
   }
 
-  using P = nvfp4::PlanPair;
-  auto kern = nvfp4::gemm_nvfp4_pair_kernel<EPI>;
+  using P = nvfp4::PlanPairT<MX>;
+  auto kern = nvfp4::gemm_nvfp4_pair_kernel<EPI, MX>;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cudaLaunchAttribute attr[1];
@@ -196,16 +200,16 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   int max_clusters;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!info->pair_attr_set[EPI]) {
+    if (!info->pair_attr_set[EPI + 4 * MX]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
         return NVFP4_ERR_CUDA;
       cfg.gridDim = dim3(2 * (info->sm_count / 2), 1, 1);
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return NVFP4_ERR_CUDA;
-      info->pair_clusters[EPI] = n;
-      info->pair_attr_set[EPI] = true;
+      info->pair_clusters[EPI + 4 * MX] = n;
+      info->pair_attr_set[EPI + 4 * MX] = true;
     }
-    max_clusters = info->pair_clusters[EPI];
+    max_clusters = info->pair_clusters[EPI + 4 * MX];
   }
   const int clusters = args.num_tiles < max_clusters ? args.num_tiles : max_clusters;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
@@ -358,6 +362,56 @@ NVFP4_API nvfp4_status gemm_nvfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, cons
     args.q_cols = static_cast<int>(B.rows);
   }
   return run_gemm<nvfp4::EPI_POINTWISE>(A, B, D, ldd, B.rows, args, stream);
+}
+
+NVFP4_API int64_t mxfp4_sf_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return -1;
+  return ((rows + 127) / 128) * 128 * ((cols / 32 + 3) / 4) * 4;
+}
+
+NVFP4_API nvfp4_status mxfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int flags,
+                                      nvfp4_tensor out, cudaStream_t stream) {
+  if (x == nullptr || out.codes == nullptr || out.sf == nullptr || out.gscale == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~MXFP4_HADAMARD32) return NVFP4_ERR_INVALID_ARG;
+  if (out.rows != rows || out.cols != cols) return NVFP4_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0 || cols % 128 != 0 || ldx < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > (1ll << 31) || cols > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || (ldx % 8) != 0 || !aligned16(out.codes) || (reinterpret_cast<uintptr_t>(out.sf) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(out.gscale) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  // the per-tensor factor a GEMM applies: 1, or 1/sqrt(32) per transformed operand
+  // (x H)(w H)^T = 32 x w^T
+  const float g = (flags & MXFP4_HADAMARD32) ? 0.17677669529663689f : 1.0f;
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t threads = rows_pad * (cols / 32);
+  nvfp4::mx_quantize_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(x), rows, cols, ldx, (flags & MXFP4_HADAMARD32) ? 1 : 0,
+      static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf), out.gscale, g);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+NVFP4_API nvfp4_status gemm_mxfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* bias, int act,
+                                            int out_dtype, void* D, int64_t ldd, cudaStream_t stream) {
+  if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (act != NVFP4_ACT_NONE && act != NVFP4_ACT_RELU) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F16 && out_dtype != NVFP4_OUT_F32)
+    return NVFP4_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return NVFP4_ERR_MISALIGNED;
+  nvfp4::GemmArgs args{};
+  args.bias = bias;
+  args.act = act;
+  args.out_kind = out_dtype;
+  return run_gemm<nvfp4::EPI_POINTWISE, true>(A, B, D, ldd, B.rows, args, stream);
+}
+
+NVFP4_API nvfp4_status gemm_mxfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd, cudaStream_t stream) {
+  return gemm_mxfp4_pointwise(A, B, nullptr, NVFP4_ACT_NONE, NVFP4_OUT_BF16, D, ldd, stream);
 }
 
 NVFP4_API nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,

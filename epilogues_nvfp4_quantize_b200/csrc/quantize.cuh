@@ -370,4 +370,77 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
   }
 }
 
+// =====================================================================================
+// MXFP4 (OCP Microscaling: E2M1 elements, one E8M0 scale per 32) with an optional fixed
+// block-local transform, the 32-point Walsh-Hadamard matrix H_2 (x) ... (x) H_2 (page
+// "KroQuant: efficient post-training quantization for diffusion transformers via
+// Kronecker-product structure": an invertible Kronecker-structured transform per block of
+// 32 activations; the pages' transforms are learned, this one is fixed). One thread per
+// block of 32; lanes 4k..4k+3 hold the 4 blocks of one scale word.
+// =====================================================================================
+__global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                          int64_t cols, int64_t ldx, int hadamard,
+                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                          float* __restrict__ gscale, float g) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *gscale = g;
+  const int64_t nb = cols >> 5;  // blocks of 32 per row (a multiple of 4)
+  const int64_t rows_pad = (rows + 127) & ~int64_t(127);
+  const int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const bool live = u < rows_pad * nb;
+  const int64_t r = live ? u / nb : 0, kb = live ? u - r * nb : 0;
+  float v[32];
+  uint32_t e = 0;
+  if (live && r < rows) {
+    const uint4* p = reinterpret_cast<const uint4*>(x + r * ldx + kb * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = __ldg(p + i);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[8 * i + 2 * k] = bf16_lo(w[k]);
+        v[8 * i + 2 * k + 1] = bf16_hi(w[k]);
+      }
+    }
+    if (hadamard) {
+      // fast Walsh-Hadamard transform, stage h maps (v[j], v[j+h]) to (a + b, a - b)
+#pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j & h) continue;
+          const float a = v[j], b = v[j + h];
+          v[j] = __fadd_rn(a, b);
+          v[j + h] = __fsub_rn(a, b);
+        }
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    uint32_t c[4] = {0u, 0u, 0u, 0u};
+    if (amax > 0.0f) {
+      // shared exponent floor(log2(amax)) - 2, clamped to [-127, 127] (a subnormal amax
+      // gives -127); scale X = 2^shared, code e = shared + 127
+      const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);
+      int shared = ex == 0 ? -127 : ex - 127 - 2;
+      shared = shared < -127 ? -127 : (shared > 127 ? 127 : shared);
+      e = static_cast<uint32_t>(shared + 127);
+      const float inv = __uint_as_float(static_cast<uint32_t>(127 - shared) << 23);  // 2^-shared, exact
+      float y[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) y[j] = __fmul_rn(v[j], inv);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) c[k] = cvt_e2m1x8(y + 8 * k);
+    }
+    *reinterpret_cast<uint4*>(codes + r * (cols >> 1) + kb * 16) = make_uint4(c[0], c[1], c[2], c[3]);
+  }
+  // the 4 blocks of a scale word sit in lanes 4k..4k+3 (nb % 4 == 0 keeps them in one row)
+  const int lane = threadIdx.x & 31;
+  uint32_t word = e << (8 * (lane & 3));
+  word |= __shfl_xor_sync(0xffffffffu, word, 1);
+  word |= __shfl_xor_sync(0xffffffffu, word, 2);
+  if (live && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(sf + sf_word_offset(r, kb, nb)) = word;
+}
+
 }  // namespace nvfp4

@@ -124,6 +124,40 @@ nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int6
                                  void* workspace, cudaStream_t stream);
 
 /*
+ * MXFP4 (OCP Microscaling: E2M1 elements, one E8M0 power-of-two scale per 32 values along
+ * the columns, no per-tensor scale) with an optional fixed block transform, the 32-point
+ * Walsh-Hadamard matrix H32 = H2 (x) H2 (x) H2 (x) H2 (x) H2 ("KroQuant: efficient
+ * post-training quantization for diffusion transformers via Kronecker-product structure":
+ * an invertible Kronecker-structured transform per block of 32; learned there, fixed here).
+ *   flags: 0, or MXFP4_HADAMARD32: quantise x H32 (per block of 32, fast Walsh-Hadamard
+ *          transform in float32) instead of x. Transform both GEMM operands: (x H)(w H)^T =
+ *          32 x w^T, which the per-tensor factor absorbs.
+ *   Per block: shared = clamp(floor(log2(amax)) - 2, -127, 127), scale code e = shared + 127,
+ *   q_i = E2M1_rn_satfinite(x_i / 2^shared); an all-zero block has e = 0 and zero codes.
+ *   out.codes: rows x cols/2 bytes; out.sf: mxfp4_sf_bytes(rows, cols) bytes in the tensor-
+ *   core scale layout counting blocks of 32 (unit = 128 rows x 4 blocks; row r, block c at
+ *   (r % 32) * 16 + (r / 32) * 4 + c); *out.gscale is set to the factor a GEMM applies: 1, or
+ *   fp32(1/sqrt(32)) with the transform.
+ * Rules: cols % 128 == 0, ldx >= cols, x and ldx*2 bytes 16-byte aligned, out.codes 16-byte
+ *        and out.sf, out.gscale 4-byte aligned.
+ */
+#define MXFP4_HADAMARD32 2
+int64_t mxfp4_sf_bytes(int64_t rows, int64_t cols);
+nvfp4_status mxfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int flags,
+                            nvfp4_tensor out, cudaStream_t stream);
+
+/*
+ * GEMM on MXFP4 operands (from mxfp4_quantize; B is N x K): as gemm_nvfp4_pointwise without
+ * the NVFP4 output, with the tensor-core MMA kind mxf4nvf4 at block32 (E8M0 scales).
+ * alpha = G_A * G_B (1, or 1/32 when both operands carry the transform).
+ */
+nvfp4_status gemm_mxfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* bias, int act,
+                                  int out_dtype, void* D, int64_t ldd, cudaStream_t stream);
+/* D = bf16(G_A G_B acc) on MXFP4 operands. */
+nvfp4_status gemm_mxfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                              cudaStream_t stream);
+
+/*
  * D (M x N bf16, leading dimension ldd) = bf16(G_A * G_B * sum_k A[m,k] * B[n,k]) with
  * A (M x K) and B (N x K) NVFP4, both K-contiguous.
  * Rules: M % 128 == 0, N % 256 == 0, K % 256 == 0, A.cols == B.cols == K,
