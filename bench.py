@@ -404,6 +404,30 @@ def run_cuda(args):
         }
         del xm, wm, c_mx, c_nv, w_up_bf16
 
+    # ---- a small-batch step (serving): eager launches vs one CUDA-graph replay
+    if not args.no_unfused:
+        small = Layer(1024, dev, seed=rank + 100)
+        barrier()
+        t_eager = time_loop(small.step, args.cmp_steps, 3, torch)
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
+            small.step()
+        torch.cuda.current_stream().wait_stream(gs)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            small.step()
+        t_graph = time_loop(graph.replay, args.cmp_steps, 3, torch)
+        fl_small = sum(step_flops(1024).values())
+        result["small_batch_graph"] = {
+            "M": 1024, "eager_us": round(t_eager * 1e3, 1), "graph_us": round(t_graph * 1e3, 1),
+            "eager_tflops": round(fl_small / (t_eager * 1e-3) / 1e12, 1),
+            "graph_tflops": round(fl_small / (t_graph * 1e-3) / 1e12, 1),
+        }
+        del graph, small
+        torch.cuda.empty_cache()
+
     # ---- fake quantisation (quantization-aware distillation forward), HBM-bound
     if not args.no_unfused:
         y_fq = torch.empty_like(layer.x)
