@@ -10,6 +10,8 @@ from ._lib import (  # noqa: F401
     NVFP4Tensor,
     gemm_mxfp4_plain,
     gemm_mxfp4_pointwise,
+    gemm_mxfp4_rmsnorm,
+    gemm_mxfp4_swiglu,
     gemm_nvfp4_plain,
     gemm_nvfp4_pointwise,
     gemm_nvfp4_rmsnorm,

@@ -26,6 +26,7 @@ EXPORTS = (
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
     "nvfp4_quantize_noalloc", "nvfp4_fake_quantize", "gemm_nvfp4_pointwise",
     "mxfp4_sf_bytes", "mxfp4_quantize", "gemm_mxfp4_pointwise", "gemm_mxfp4_plain",
+    "gemm_mxfp4_rmsnorm", "gemm_mxfp4_swiglu",
 )
 
 
@@ -66,6 +67,8 @@ def load() -> ctypes.CDLL:
         "mxfp4_quantize": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
         "gemm_mxfp4_pointwise": (i32, [_Tensor, _Tensor, vp, i32, i32, vp, i64, vp]),
         "gemm_mxfp4_plain": (i32, [_Tensor, _Tensor, vp, i64, vp]),
+        "gemm_mxfp4_rmsnorm": (i32, [_Tensor, _Tensor, vp, i32, i64, f32, vp, i64, vp]),
+        "gemm_mxfp4_swiglu": (i32, [_Tensor, _Tensor, vp, i64, ctypes.POINTER(_Tensor), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -196,14 +199,35 @@ def gemm_nvfp4_pointwise(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tenso
 MXFP4_HADAMARD32 = 2
 
 
-def mxfp4_quantize(x: torch.Tensor, out: NVFP4Tensor, hadamard: bool = False, stream=None) -> NVFP4Tensor:
+def mxfp4_quantize(x: torch.Tensor, out: NVFP4Tensor, hadamard: bool = False, interleave: bool = False,
+                   stream=None) -> NVFP4Tensor:
     """MXFP4-quantise a bf16 2-D CUDA tensor (optionally after the 32-point block Hadamard
-    transform) into `out` (from NVFP4Tensor.empty_mx); see mxfp4_quantize in the header."""
+    transform, optionally with the SwiGLU gate/up row interleave) into `out` (from
+    NVFP4Tensor.empty_mx); see mxfp4_quantize in the header."""
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
-    _check(load().mxfp4_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0),
-                                 MXFP4_HADAMARD32 if hadamard else 0, out.c(), _stream(stream)), "mxfp4_quantize")
+    flags = (MXFP4_HADAMARD32 if hadamard else 0) | (SWIGLU_INTERLEAVE if interleave else 0)
+    _check(load().mxfp4_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), flags, out.c(),
+                                 _stream(stream)), "mxfp4_quantize")
     return out
+
+
+def gemm_mxfp4_rmsnorm(A: NVFP4Tensor, B: NVFP4Tensor, w: Optional[torch.Tensor], head_dim: int,
+                       n_norm_cols: int, eps: float, D: torch.Tensor, stream=None) -> torch.Tensor:
+    if w is not None and (w.dtype != torch.float32 or not w.is_contiguous()):
+        raise ValueError("w must be a contiguous float32 tensor")
+    p, ld = _out2d(D)
+    _check(load().gemm_mxfp4_rmsnorm(A.c(), B.c(), _ptr(w), head_dim, n_norm_cols, eps, p, ld, _stream(stream)),
+           "gemm_mxfp4_rmsnorm")
+    return D
+
+
+def gemm_mxfp4_swiglu(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tensor] = None,
+                      Dq: Optional[NVFP4Tensor] = None, stream=None):
+    p, ld = _out2d(D)
+    dq = ctypes.pointer(Dq.c()) if Dq is not None else None
+    _check(load().gemm_mxfp4_swiglu(A.c(), B.c(), p, ld, dq, _stream(stream)), "gemm_mxfp4_swiglu")
+    return D, Dq
 
 
 def gemm_mxfp4_pointwise(A: NVFP4Tensor, B: NVFP4Tensor, D: torch.Tensor, bias: Optional[torch.Tensor] = None,

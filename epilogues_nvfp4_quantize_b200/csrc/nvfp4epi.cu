@@ -373,7 +373,8 @@ NVFP4_API nvfp4_status mxfp4_quantize(const void* x, int64_t rows, int64_t cols,
                                       nvfp4_tensor out, cudaStream_t stream) {
   if (x == nullptr || out.codes == nullptr || out.sf == nullptr || out.gscale == nullptr)
     return NVFP4_ERR_INVALID_ARG;
-  if (flags & ~MXFP4_HADAMARD32) return NVFP4_ERR_INVALID_ARG;
+  if (flags & ~(MXFP4_HADAMARD32 | NVFP4_SWIGLU_INTERLEAVE)) return NVFP4_ERR_INVALID_ARG;
+  if ((flags & NVFP4_SWIGLU_INTERLEAVE) && (rows % 2) != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (out.rows != rows || out.cols != cols) return NVFP4_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0 || cols % 128 != 0 || ldx < cols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (rows > (1ll << 31) || cols > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -391,6 +392,7 @@ NVFP4_API nvfp4_status mxfp4_quantize(const void* x, int64_t rows, int64_t cols,
   const int64_t threads = rows_pad * (cols / 32);
   nvfp4::mx_quantize_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
       static_cast<const uint16_t*>(x), rows, cols, ldx, (flags & MXFP4_HADAMARD32) ? 1 : 0,
+      (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0,
       static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf), out.gscale, g);
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
@@ -414,9 +416,9 @@ NVFP4_API nvfp4_status gemm_mxfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D,
   return gemm_mxfp4_pointwise(A, B, nullptr, NVFP4_ACT_NONE, NVFP4_OUT_BF16, D, ldd, stream);
 }
 
-NVFP4_API nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,
-                                          int64_t n_norm_cols, float eps, void* D, int64_t ldd,
-                                          cudaStream_t stream) {
+template <bool MX>
+static nvfp4_status rmsnorm_entry(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim, int64_t n_norm_cols,
+                                  float eps, void* D, int64_t ldd, cudaStream_t stream) {
   if (D == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (head_dim != 128 && head_dim != 256) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (n_norm_cols < 0 || n_norm_cols > B.rows || n_norm_cols % head_dim != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -428,11 +430,24 @@ NVFP4_API nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const 
   args.head_dim = head_dim;
   args.n_norm_cols = static_cast<int>(n_norm_cols);
   args.eps = eps;
-  return run_gemm<nvfp4::EPI_RMSNORM>(A, B, D, ldd, B.rows, args, stream);
+  return run_gemm<nvfp4::EPI_RMSNORM, MX>(A, B, D, ldd, B.rows, args, stream);
 }
 
-NVFP4_API nvfp4_status gemm_nvfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
-                                         const nvfp4_tensor* Dq, cudaStream_t stream) {
+NVFP4_API nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,
+                                          int64_t n_norm_cols, float eps, void* D, int64_t ldd,
+                                          cudaStream_t stream) {
+  return rmsnorm_entry<false>(A, B, w, head_dim, n_norm_cols, eps, D, ldd, stream);
+}
+
+NVFP4_API nvfp4_status gemm_mxfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,
+                                          int64_t n_norm_cols, float eps, void* D, int64_t ldd,
+                                          cudaStream_t stream) {
+  return rmsnorm_entry<true>(A, B, w, head_dim, n_norm_cols, eps, D, ldd, stream);
+}
+
+template <bool MX>
+static nvfp4_status swiglu_entry(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd, const nvfp4_tensor* Dq,
+                                 cudaStream_t stream) {
   if (D == nullptr && Dq == nullptr) return NVFP4_ERR_INVALID_ARG;
   const int64_t nh = B.rows / 2;
   nvfp4::GemmArgs args{};
@@ -445,7 +460,17 @@ NVFP4_API nvfp4_status gemm_nvfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D
     args.q_gscale = Dq->gscale;
     args.q_cols = static_cast<int>(nh);
   }
-  return run_gemm<nvfp4::EPI_SWIGLU>(A, B, D, ldd, nh, args, stream);
+  return run_gemm<nvfp4::EPI_SWIGLU, MX>(A, B, D, ldd, nh, args, stream);
+}
+
+NVFP4_API nvfp4_status gemm_nvfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                                         const nvfp4_tensor* Dq, cudaStream_t stream) {
+  return swiglu_entry<false>(A, B, D, ldd, Dq, stream);
+}
+
+NVFP4_API nvfp4_status gemm_mxfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                                         const nvfp4_tensor* Dq, cudaStream_t stream) {
+  return swiglu_entry<true>(A, B, D, ldd, Dq, stream);
 }
 
 NVFP4_API nvfp4_status rmsnorm_heads_bf16(const void* x, int64_t rows, int64_t ldx, const float* w, int head_dim,

@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
 // block of 32; lanes 4k..4k+3 hold the 4 blocks of one scale word.
 // =====================================================================================
 __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                          int64_t cols, int64_t ldx, int hadamard,
+                                                          int64_t cols, int64_t ldx, int hadamard, int interleave,
                                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                           float* __restrict__ gscale, float g) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *gscale = g;
@@ -391,7 +391,9 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
   float v[32];
   uint32_t e = 0;
   if (live && r < rows) {
-    const uint4* p = reinterpret_cast<const uint4*>(x + r * ldx + kb * 32);
+    // with `interleave`, output row 2j reads input row j and 2j+1 reads input row rows/2 + j
+    const int64_t src = interleave ? ((r & 1) ? (rows >> 1) + (r >> 1) : (r >> 1)) : r;
+    const uint4* p = reinterpret_cast<const uint4*>(x + src * ldx + kb * 32);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint4 q = __ldg(p + i);

@@ -129,9 +129,10 @@ nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int6
  * Walsh-Hadamard matrix H32 = H2 (x) H2 (x) H2 (x) H2 (x) H2 ("KroQuant: efficient
  * post-training quantization for diffusion transformers via Kronecker-product structure":
  * an invertible Kronecker-structured transform per block of 32; learned there, fixed here).
- *   flags: 0, or MXFP4_HADAMARD32: quantise x H32 (per block of 32, fast Walsh-Hadamard
+ *   flags: MXFP4_HADAMARD32: quantise x H32 (per block of 32, fast Walsh-Hadamard
  *          transform in float32) instead of x. Transform both GEMM operands: (x H)(w H)^T =
- *          32 x w^T, which the per-tensor factor absorbs.
+ *          32 x w^T, which the per-tensor factor absorbs. NVFP4_SWIGLU_INTERLEAVE: the row
+ *          permutation of a [gate | up] weight, as for nvfp4_quantize (rows even).
  *   Per block: shared = clamp(floor(log2(amax)) - 2, -127, 127), scale code e = shared + 127,
  *   q_i = E2M1_rn_satfinite(x_i / 2^shared); an all-zero block has e = 0 and zero codes.
  *   out.codes: rows x cols/2 bytes; out.sf: mxfp4_sf_bytes(rows, cols) bytes in the tensor-
@@ -156,6 +157,14 @@ nvfp4_status gemm_mxfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* b
 /* D = bf16(G_A G_B acc) on MXFP4 operands. */
 nvfp4_status gemm_mxfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
                               cudaStream_t stream);
+/* gemm_nvfp4_rmsnorm and gemm_nvfp4_swiglu on MXFP4 operands (same arguments and rules; the
+ * SwiGLU weight is packed with mxfp4_quantize(..., NVFP4_SWIGLU_INTERLEAVE | ...), and the
+ * optional re-quantised output Dq is NVFP4). */
+nvfp4_status gemm_mxfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w, int head_dim,
+                                int64_t n_norm_cols, float eps, void* D, int64_t ldd,
+                                cudaStream_t stream);
+nvfp4_status gemm_mxfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,
+                               const nvfp4_tensor* Dq, cudaStream_t stream);
 
 /*
  * D (M x N bf16, leading dimension ldd) = bf16(G_A * G_B * sum_k A[m,k] * B[n,k]) with

@@ -97,3 +97,44 @@ def test_mx_gemm_with_transform_matches_oracle_and_beats_no_transform_on_outlier
         errs[hadamard] = np.linalg.norm(got - exact) / np.linalg.norm(exact)
     assert errs[True] < errs[False], errs
     assert ep.read_device_status() == 0
+
+
+def test_mx_quantize_interleaved_weight_bitwise():
+    w = wk.weights(2 * 200, 256, 1 / 16, seed=21)
+    t = ep.mxfp4_quantize(w.to(device()), ep.NVFP4Tensor.empty_mx(400, 256, device()), hadamard=True, interleave=True)
+    q_ref, e_ref = o.mx_quantize(o.hadamard32(o.interleave_gate_up(w.float().numpy())))
+    q, e, _, _ = _read_mx(t)
+    assert np.array_equal(e, e_ref) and np.array_equal(q, q_ref)
+
+
+@pytest.mark.parametrize("M,hd", [(256, 256), (384, 128)])
+def test_mx_rmsnorm_gemm_matches_oracle(M, hd):
+    K, N, n_norm = 1024, 1024, 512
+    a = wk.activations(M, K, 2, seed=M)
+    b = wk.weights(N, K, 1 / np.sqrt(K), seed=M + 1)
+    w = np.tile(wk.norm_weight(hd, 0, 3), n_norm // hd).astype(np.float32)
+    A = ep.mxfp4_quantize(a.to(device()), ep.NVFP4Tensor.empty_mx(M, K, device()), hadamard=True)
+    B = ep.mxfp4_quantize(b.to(device()), ep.NVFP4Tensor.empty_mx(N, K, device()), hadamard=True)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    ep.gemm_mxfp4_rmsnorm(A, B, torch.from_numpy(w).to(device()), hd, n_norm, 1e-6, D)
+    g = float(np.float32(1 / np.sqrt(32)))
+    c = g * g * o.gemm(o.mx_dequantize(*o.mx_quantize(o.hadamard32(a.float().numpy()))),
+                       o.mx_dequantize(*o.mx_quantize(o.hadamard32(b.float().numpy()))))
+    ref = o.bf16_round(o.rmsnorm_heads(c, w, hd, n_norm, 1e-6))
+    assert_close(D.float().cpu().numpy().astype(np.float64), ref, "mxfp4 rmsnorm")
+
+
+def test_mx_swiglu_gemm_matches_oracle():
+    M, K, nh = 256, 512, 512
+    a = wk.activations(M, K, 2, seed=3)
+    b = wk.weights(2 * nh, K, 1 / np.sqrt(K), seed=4)
+    A = ep.mxfp4_quantize(a.to(device()), ep.NVFP4Tensor.empty_mx(M, K, device()), hadamard=True)
+    B = ep.mxfp4_quantize(b.to(device()), ep.NVFP4Tensor.empty_mx(2 * nh, K, device()), hadamard=True, interleave=True)
+    D = torch.empty(M, nh, dtype=torch.bfloat16, device=device())
+    ep.gemm_mxfp4_swiglu(A, B, D)
+    g = float(np.float32(1 / np.sqrt(32)))
+    c = g * g * o.gemm(o.mx_dequantize(*o.mx_quantize(o.hadamard32(a.float().numpy()))),
+                       o.mx_dequantize(*o.mx_quantize(o.hadamard32(b.float().numpy()))))
+    ref = o.bf16_round(o.swiglu(c))
+    assert_close(D.float().cpu().numpy().astype(np.float64), ref, "mxfp4 swiglu")
+    assert ep.read_device_status() == 0
