@@ -12,15 +12,24 @@
 //   gemm_nvfp4_kernel       (M % 256 == 128) one CTA per 128 x 256 tile (3-stage ring).
 // Warp roles (384 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
 // and MMA issuer, warps 10-11 copy the block scales from shared memory into TMEM
-// (tcgen05.cp). Each tcgen05 instruction holds up the warp that issues it for a while;
-// issued from their own warps (on other SM sub-partitions) the 12 scale copies of a K step
-// overlap the 4 MMAs instead of queueing in front of them. Two TMEM scale slots let the
-// copies of K step g+1 run while the MMAs of step g read the other slot.
+// (tcgen05.cp).
+// Issue cost sets the main loop's pace. A tcgen05.mma holds up its issuing thread for
+// about as long as the tensor pipe takes to run it (M 256 x N 256 x K 64: 128 cycles),
+// so the pipe holds no backlog. Whatever else that thread does between two K steps leaves
+// the pipe idle. So the MMA thread does only this per K step: one wait on the stage's
+// barrier, the 4 MMAs and one commit that frees the stage.
+// - The scale copies are issued from their own warps, on other SM sub-partitions.
+// - The copy warps' commits land on the same stage barrier as the operand bytes, so one
+//   wait covers the operand tiles and the scales.
+// - A scale slot in TMEM is free again once the stage-empty commit of the step that last
+//   used it has arrived.
+// - NSLOT (3 or 4) slots let the copies run ahead of the MMAs by NSLOT - 1 steps.
+// TMEM holds one 256-column FP32 accumulator at column 0 and the scale slots behind it.
+// The MMAs of tile i+1 start once both epilogue warpgroups have moved tile i's
+// accumulator into registers.
 // Epilogue warp w reads TMEM lanes 32*(w%4).. (its 32 output rows) and columns
 // 128*(w/4).. (its half of the 256-column tile); each thread owns one output row.
-// Results go through a 128-byte-swizzled staging box and a TMA store. Two accumulator
-// buffers in TMEM let the MMAs of tile i+1 run while the epilogue of tile i reads its
-// buffer.
+// Results go through a 128-byte-swizzled staging box and a TMA store.
 //
 // Epilogues:
 //   PLAIN    y = alpha * acc,  alpha = G_A * G_B
@@ -67,18 +76,14 @@ constexpr int COPY_WARP0 = EPI_WARPS + 2;
 constexpr int BOX_BYTES = 32 * 128;     // one staging box: 32 rows x 128 bytes
 constexpr int RED_BYTES = 2 * 2 * 128 * 4;
 constexpr uint32_t TMEM_COLS = 512;
-// Two 256-column FP32 accumulators that overlap in 96 columns, so that both fit beside two
-// 48-column slots of block scales: buffer 0 = [0, 256), buffer 1 = [160, 416), scale slots
-// at 416 and 464. The overlap [160, 256) is held by warpgroup 1 of buffer 0 and warpgroup 0
-// of buffer 1; the next tile may start once that warpgroup has read its columns.
-constexpr uint32_t ACC_COL1 = 160;
-constexpr uint32_t SF_SLOT0 = 416;
+// The FP32 accumulator takes columns [0, 256); the block scales of one K step take a
+// 48-column slot behind it, up to 5 slots (the kernels use 3 or 4).
+constexpr uint32_t SF_SLOT0 = 256;
 constexpr uint32_t SF_SLOT_COLS = 48;  // per K step: SFA 4 MMAs x 4 columns, then SFB 4 MMAs x 8
 constexpr uint32_t SFB_OFF = 16;
-__host__ __device__ constexpr uint32_t acc_col(uint32_t buf) { return buf ? ACC_COL1 : 0u; }
-__host__ __device__ constexpr int overlap_wg(uint32_t buf) { return buf ? 0 : 1; }
+constexpr int MAX_SLOTS = 5;
 __host__ __device__ constexpr uint32_t sf_slot(uint32_t s) { return SF_SLOT0 + SF_SLOT_COLS * s; }
-static_assert(ACC_COL1 + 256 <= SF_SLOT0 && ACC_COL1 >= 128 && sf_slot(2) <= TMEM_COLS, "TMEM plan");
+static_assert(sf_slot(MAX_SLOTS) <= TMEM_COLS, "TMEM plan");
 }  // namespace gemm_cfg
 
 // Block-scale format: NVFP4 (E4M3 scale per 16 values) or MXFP4 (E8M0 scale per 32). A
@@ -100,7 +105,7 @@ struct SmemPlan {
   static constexpr int OFF_EPI = S * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
   static constexpr int OFF_BAR = OFF_RED + gemm_cfg::RED_BYTES;
-  static constexpr int NUM_BARS = 3 * S + 14;  // full, empty, 14 more (bar_idx), scales loaded
+  static constexpr int NUM_BARS = 3 * S + 7;  // full, empty, 7 more (bar_idx), scales loaded
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -114,39 +119,35 @@ using PlanSingle = PlanSingleT<false>;
 using PlanPair = PlanPairT<false>;
 
 // Barriers past the stage ring (full[S], empty[S]), at empty + S + index.
+//   full[s]:  the stage's operand bytes (expect-tx arrival) and one commit per copy warp
+//             once the stage's scales are in TMEM
+//   empty[s]: one MMA commit when the stage's MMAs are done (frees the stage and the scale
+//             slot its step used)
 namespace bar_idx {
-constexpr int ACC_FULL = 0;   // [2]
-constexpr int ACC_EMPTY = 2;  // [2][2]
-constexpr int RED = 6;
-constexpr int DRAIN = 7;      // MMA warp's own drain on give-up
-constexpr int SF_FULL = 8;    // [2] scale slot filled (one commit per copy warp)
-constexpr int SF_EMPTY = 10;  // [2] scale slot read by the MMAs (one MMA commit)
-constexpr int CP_DRAIN = 12;  // [COPY_WARPS] copy warps' own drain on give-up
-constexpr int SF_LOADED = 14; // [S] a stage's scale units have landed (their own tx count)
+constexpr int ACC_FULL = 0;   // MMA commit: the tile's accumulator is complete
+constexpr int ACC_EMPTY = 1;  // [2] per epilogue warpgroup: accumulator moved to registers
+constexpr int RED = 3;
+constexpr int DRAIN = 4;      // MMA warp's own drain on give-up
+constexpr int CP_DRAIN = 5;   // [COPY_WARPS] copy warps' own drain on give-up
+constexpr int SF_LOADED = 7;  // [S] a stage's scale units have landed (their own tx count)
 }  // namespace bar_idx
-static_assert(bar_idx::CP_DRAIN + gemm_cfg::COPY_WARPS <= 14, "barrier plan");
+static_assert(bar_idx::CP_DRAIN + gemm_cfg::COPY_WARPS <= bar_idx::SF_LOADED, "barrier plan");
 
-// Accumulator hand-off between the MMA warp and the epilogue: per buffer one "full"
-// barrier (MMA commit) and one "empty" barrier per warpgroup (one arrival per warp of that
-// warpgroup, in each CTA of the pair).
+// Accumulator hand-off between the MMA warp and the epilogue: one "full" barrier (MMA
+// commit) and one "empty" barrier per warpgroup (one arrival per warp of that warpgroup,
+// in each CTA of the pair).
 struct AccBars {
-  uint64_t* full;   // [2]
-  uint64_t* empty;  // [2][2]: empty[2 * buf + wg]
-  __device__ __forceinline__ uint64_t* emp(uint32_t buf, int wg) const { return empty + 2 * buf + wg; }
+  uint64_t* full;
+  uint64_t* empty;  // [2]: empty[wg]
+  __device__ __forceinline__ uint64_t* emp(int wg) const { return empty + wg; }
 };
 
-// MMA side: before tile j (buffer j & 1) may overwrite its accumulator, both warpgroups
-// must have read the buffer's previous tile (j - 2), and the warpgroup holding the
-// overlap must have read tile j - 1 (the other buffer).
+// MMA side: tile j may overwrite the accumulator once both warpgroups have read tile j - 1.
 __device__ __forceinline__ bool acc_acquire(const AccBars& a, uint32_t j, volatile int* abort_flag,
                                             uint64_t limit, int where) {
-  const uint32_t b = j & 1u, u = j >> 1;
-  if (!mbar_wait(a.emp(b, 0), (u & 1u) ^ 1u, abort_flag, limit, where)) return false;
-  if (!mbar_wait(a.emp(b, 1), (u & 1u) ^ 1u, abort_flag, limit, where)) return false;
-  if (j >= 1) {
-    const uint32_t bp = b ^ 1u, up = (j - 1) >> 1;
-    if (!mbar_wait(a.emp(bp, gemm_cfg::overlap_wg(bp)), up & 1u, abort_flag, limit, where)) return false;
-  }
+  const uint32_t parity = (j & 1u) ^ 1u;
+  if (!mbar_wait(a.emp(0), parity, abort_flag, limit, where)) return false;
+  if (!mbar_wait(a.emp(1), parity, abort_flag, limit, where)) return false;
   return true;
 }
 
@@ -156,30 +157,38 @@ __device__ __forceinline__ uint32_t ksteps_of(int num_tiles, int K, int first, i
   return static_cast<uint32_t>(tiles) * static_cast<uint32_t>(K / gemm_cfg::BK);
 }
 
-// Scale-copy warp `cw` (one elected lane). For K step g in stage `stage`: once the stage's
-// scale units have landed (they have their own barrier, so the copies overlap the arrival
-// of the larger code tiles) and the MMAs of step g - 2 have finished reading scale slot g % 2, copy its
-// share of the step's scale units (12 for NVFP4, 6 for MXFP4; unit i goes to warp
-// i % COPY_WARPS) into that slot and commit to sf_full[g % 2]. Slot layout: SFA unit q at
-// columns 4q, SFB rows 0-127 of unit q at 16 + 8q, rows 128-255 at 16 + 8q + 4. An NVFP4
-// unit serves one K = 64 MMA; an MXFP4 unit two (bytes 0-1 and 2-3 of each word). In a CTA pair the leader copies for both CTAs and
-// the commits go to the leader's barriers only. Returns false if a bounded wait gave up
-// (after waiting, bounded, for its own copies).
-template <bool PAIR, bool MX, int STAGES, int STAGE_BYTES, int SF_OFF, int SFB_HALF>
-__device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* bars, uint32_t tmem,
+// Scale-copy warp `cw` (one elected lane), K step g in ring stage `stage`, scale slot
+// g % NSLOT.
+// 1. Wait until the stage's scale units have landed. They have their own barrier, so the
+//    copies overlap the arrival of the larger code tiles.
+// 2. Wait until the slot is free, i.e. the stage-empty commit of step g - NSLOT has
+//    arrived. Parity waits on that barrier stay unambiguous while NSLOT <= STAGES: its
+//    next completion belongs to step g - NSLOT + STAGES >= g, whose MMAs cannot finish
+//    before this step's copies.
+// 3. Copy this warp's share of the step's scale units into the slot: 12 units for NVFP4,
+//    6 for MXFP4; unit i goes to warp i % COPY_WARPS.
+// 4. Commit onto the stage's operand barrier, so that the MMA warp's single wait covers the
+//    scales too.
+// Slot layout: SFA unit q at columns 4q, SFB rows 0-127 of unit q at 16 + 8q, rows
+// 128-255 at 16 + 8q + 4. An NVFP4 unit serves one K = 64 MMA; an MXFP4 unit two (bytes 0-1
+// and 2-3 of each word).
+// In a CTA pair the leader copies for both CTAs, and the commits go to the leader's
+// barriers only. Returns false if a bounded wait gave up, after waiting (bounded) for its
+// own copies.
+template <bool PAIR, bool MX, int STAGES, int NSLOT, int STAGE_BYTES, int SF_OFF, int SFB_HALF>
+__device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* full, uint64_t* bars, uint32_t tmem,
                                                 int cw, uint32_t nsteps, volatile int* abort_flag, uint64_t limit,
                                                 int where) {
   using namespace gemm_cfg;
-  uint64_t* sf_full = bars + bar_idx::SF_FULL;
-  uint64_t* sf_empty = bars + bar_idx::SF_EMPTY;
+  static_assert(NSLOT >= 2 && NSLOT <= STAGES && NSLOT <= MAX_SLOTS, "scale slots");
+  uint64_t* empty = full + STAGES;
   uint64_t* sf_loaded = bars + bar_idx::SF_LOADED;
-  int stage = 0;
-  uint32_t phase = 0;
+  int stage = 0, slot_i = 0, reuse = 0;  // reuse: stage of step g - NSLOT
+  uint32_t phase = 0, reuse_phase = 0;
   bool ok = true;
   for (uint32_t g = 0; g < nsteps; ++g) {
-    const uint32_t s = g & 1u, u = g >> 1;
     if (!mbar_wait(&sf_loaded[stage], phase, abort_flag, limit, where) ||
-        !mbar_wait(&sf_empty[s], (u & 1u) ^ 1u, abort_flag, limit, where + 1)) {
+        (g >= static_cast<uint32_t>(NSLOT) && !mbar_wait(&empty[reuse], reuse_phase, abort_flag, limit, where + 1))) {
       ok = false;
       break;
     }
@@ -187,7 +196,7 @@ __device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* bars, u
     constexpr int U = ScaleFmt<MX>::UNITS;
     const uint32_t sfa = smem_u32(smem + stage * STAGE_BYTES) + SF_OFF;
     const uint32_t sfb = sfa + U * SF_UNIT;
-    const uint32_t slot = tmem + sf_slot(s);
+    const uint32_t slot = tmem + sf_slot(slot_i);
 #pragma unroll
     for (int i = 0; i < 3 * U; ++i) {
       if (i % COPY_WARPS != cw) continue;
@@ -201,22 +210,23 @@ __device__ __forceinline__ bool scale_copy_loop(uint8_t* smem, uint64_t* bars, u
       }
     }
     if constexpr (PAIR) {
-      tc_commit_pair(&sf_full[s], 0x1);
+      tc_commit_pair(&full[stage], 0x1);
     } else {
-      tc_commit(&sf_full[s]);
+      tc_commit(&full[stage]);
     }
     if (++stage == STAGES) {
       stage = 0;
       phase ^= 1u;
     }
-  }
-  if (ok) {
-    // Tail: wait for the MMA commits that release the last two slots, so that no arrival
-    // reaches this CTA's barriers after it exits.
-    for (uint32_t g = nsteps; g < nsteps + 2; ++g) {
-      if (!mbar_wait(&sf_empty[g & 1u], ((g >> 1) & 1u) ^ 1u, abort_flag, limit, where + 1)) break;
+    if (++slot_i == NSLOT) slot_i = 0;
+    if (g >= static_cast<uint32_t>(NSLOT)) {  // the next step reuses the slot of step g + 1 - NSLOT
+      if (++reuse == STAGES) {
+        reuse = 0;
+        reuse_phase ^= 1u;
+      }
     }
-  } else {
+  }
+  if (!ok) {
     uint64_t* drain = bars + bar_idx::CP_DRAIN + cw;
     if constexpr (PAIR) {
       tc_commit_pair(drain, 0x1);
@@ -310,11 +320,11 @@ struct EpiCtx {
 // start the next tile while the op, the rounding and the stores run. Returns false if a
 // bounded wait gave up.
 template <int EPI, class Release>
-__device__ __forceinline__ bool epilogue_tile(EpiCtx& c, uint32_t buf, int m0, int n0, Release release) {
+__device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release release) {
   using namespace gemm_cfg;
   const GemmArgs& args = *c.args;
   const int lane = c.lane;
-  const uint32_t tcol = c.t_row + acc_col(buf) + c.wg * 128;
+  const uint32_t tcol = c.t_row + c.wg * 128;
   const int col0 = n0 + c.wg * 128;
   const int row_in_tile = c.sub * 32 + lane;
   const float alpha = c.alpha;
@@ -531,14 +541,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   using P = PlanSingleT<MX>;
   constexpr int U = ScaleFmt<MX>::UNITS;
   constexpr int STAGES = 3;
+  constexpr int NSLOT = 3;  // scale slots in TMEM (at most STAGES)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* empty = full + STAGES;
-  AccBars acc{empty + STAGES, empty + STAGES + 2};
-  uint64_t* red_bar = empty + STAGES + 6;
-  uint64_t* drain_bar = empty + STAGES + 7;
   uint64_t* xbars = empty + STAGES;  // bar_idx layout
+  AccBars acc{xbars + bar_idx::ACC_FULL, xbars + bar_idx::ACC_EMPTY};
+  uint64_t* red_bar = xbars + bar_idx::RED;
+  uint64_t* drain_bar = xbars + bar_idx::DRAIN;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
@@ -548,20 +559,14 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + COPY_WARPS);  // expect-tx arrival, then one commit per copy warp
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc.full[b], 1);
-      mbar_init(acc.emp(b, 0), EPI_WARPS / 2);
-      mbar_init(acc.emp(b, 1), EPI_WARPS / 2);
-    }
+    mbar_init(acc.full, 1);
+    mbar_init(acc.emp(0), EPI_WARPS / 2);
+    mbar_init(acc.emp(1), EPI_WARPS / 2);
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&xbars[bar_idx::SF_FULL + b], COPY_WARPS);
-      mbar_init(&xbars[bar_idx::SF_EMPTY + b], 1);
-    }
     for (int w = 0; w < COPY_WARPS; ++w) mbar_init(&xbars[bar_idx::CP_DRAIN + w], 1);
     for (int st = 0; st < STAGES; ++st) mbar_init(&xbars[bar_idx::SF_LOADED + st], 1);
     *abort_flag = 0;
@@ -646,7 +651,8 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc = MX ? idesc_mxfp4(BM, BN, 0) : idesc_nvfp4(BM, BN);
       int stage = 0;
-      uint32_t phase = 0, j = 0, g = 0;
+      uint32_t phase = 0, j = 0;
+      int sl = 0;  // scale slot of this K step
       bool ok = true;
       for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++j) {
         if (!acc_acquire(acc, j, abort_flag, limit, 2)) {
@@ -654,11 +660,9 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc_col(j & 1u);
-        for (int kt = 0; kt < ktiles; ++kt, ++g) {
-          const uint32_t sl = g & 1u;
-          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3) ||
-              !mbar_wait(&xbars[bar_idx::SF_FULL + sl], (g >> 1) & 1u, abort_flag, limit, 5)) {
+        const uint32_t d_tmem = tmem;
+        for (int kt = 0; kt < ktiles; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3)) {
             ok = false;
             break;
           }
@@ -677,14 +681,14 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
                              (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
-          tc_commit(&xbars[bar_idx::SF_EMPTY + sl]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
+          if (++sl == NSLOT) sl = 0;
         }
         if (!ok) break;
-        tc_commit(&acc.full[j & 1u]);
+        tc_commit(acc.full);
       }
       if (!ok) {
         tc_commit(drain_bar);
@@ -694,8 +698,8 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else if (warp >= COPY_WARP0) {
     // ------------------------------------------------------------------ scale copies
     if (lane == 0) {
-      (void)scale_copy_loop<false, MX, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
-          smem, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
+      (void)scale_copy_loop<false, MX, STAGES, NSLOT, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
           abort_flag, limit, 14);
     }
   } else {
@@ -705,16 +709,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, ++j) {
       int tm, tn;
       tile_coords(args, t, tm, tn);
-      const uint32_t b = j & 1u;
       auto release = [&]() {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc.emp(b, c.wg));
+        if (lane == 0) mbar_arrive(acc.emp(c.wg));
       };
       // every lane waits; the warp leaves together if any lane gave up
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc.full[b], (j >> 1) & 1u, abort_flag, limit, 4))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc.full, j & 1u, abort_flag, limit, 4))) break;
       tc_fence_after();
-      if (!epilogue_tile<EPI>(c, b, tm * BM, tn * BN, release)) break;
+      if (!epilogue_tile<EPI>(c, tm * BM, tn * BN, release)) break;
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -741,14 +744,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   using P = PlanPairT<MX>;
   constexpr int U = ScaleFmt<MX>::UNITS;
   constexpr int STAGES = 5;
+  constexpr int NSLOT = 4;  // scale slots in TMEM (at most STAGES)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* empty = full + STAGES;
-  AccBars acc{empty + STAGES, empty + STAGES + 2};  // leader's empty barriers count both CTAs
-  uint64_t* red_bar = empty + STAGES + 6;
-  uint64_t* drain_bar = empty + STAGES + 7;
   uint64_t* xbars = empty + STAGES;  // bar_idx layout
+  AccBars acc{xbars + bar_idx::ACC_FULL, xbars + bar_idx::ACC_EMPTY};  // leader's empty barriers count both CTAs
+  uint64_t* red_bar = xbars + bar_idx::RED;
+  uint64_t* drain_bar = xbars + bar_idx::DRAIN;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_MISC + 4);
 
@@ -762,20 +766,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);   // leader's: one expect-tx arrival, both CTAs' bytes
+      // leader's: one expect-tx arrival for both CTAs' bytes, then one commit per copy warp
+      mbar_init(&full[s], 1 + COPY_WARPS);
       mbar_init(&empty[s], 1);  // one multicast commit per use
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc.full[b], 1);
-      mbar_init(acc.emp(b, 0), EPI_WARPS);  // leader's: one arrival per warp of the warpgroup, per CTA
-      mbar_init(acc.emp(b, 1), EPI_WARPS);
-    }
+    mbar_init(acc.full, 1);
+    mbar_init(acc.emp(0), EPI_WARPS);  // leader's: one arrival per warp of the warpgroup, per CTA
+    mbar_init(acc.emp(1), EPI_WARPS);
     mbar_init(red_bar, EPI_THREADS);
     mbar_init(drain_bar, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&xbars[bar_idx::SF_FULL + b], COPY_WARPS);  // leader's: the leader's copy warps
-      mbar_init(&xbars[bar_idx::SF_EMPTY + b], 1);
-    }
     for (int w = 0; w < COPY_WARPS; ++w) mbar_init(&xbars[bar_idx::CP_DRAIN + w], 1);
     for (int st = 0; st < STAGES; ++st) mbar_init(&xbars[bar_idx::SF_LOADED + st], 1);
     *abort_flag = 0;
@@ -868,7 +867,8 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     if (leader && lane == 0) {
       const uint32_t idesc = MX ? idesc_mxfp4(2 * BM, BN, 0) : idesc_nvfp4(2 * BM, BN);
       int stage = 0;
-      uint32_t phase = 0, j = 0, g = 0;
+      uint32_t phase = 0, j = 0;
+      int sl = 0;  // scale slot of this K step
       bool ok = true;
       for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters, ++j) {
         if (!acc_acquire(acc, j, abort_flag, limit, 22)) {
@@ -876,11 +876,9 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc_col(j & 1u);
-        for (int kt = 0; kt < ktiles; ++kt, ++g) {
-          const uint32_t sl = g & 1u;
-          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25) ||
-              !mbar_wait(&xbars[bar_idx::SF_FULL + sl], (g >> 1) & 1u, abort_flag, limit, 28)) {
+        const uint32_t d_tmem = tmem;
+        for (int kt = 0; kt < ktiles; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25)) {
             ok = false;
             break;
           }
@@ -898,14 +896,14 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
                                   (kt > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
-          tc_commit_pair(&xbars[bar_idx::SF_EMPTY + sl], 0x1);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
+          if (++sl == NSLOT) sl = 0;
         }
         if (!ok) break;
-        tc_commit_pair(&acc.full[j & 1u], 0x3);
+        tc_commit_pair(acc.full, 0x3);
       }
       if (!ok) {
         tc_commit_pair(drain_bar, 0x1);
@@ -915,8 +913,8 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   } else if (warp >= COPY_WARP0) {
     // ------------------------------------------------------------------ scale copies (leader only)
     if (leader && lane == 0) {
-      (void)scale_copy_loop<true, MX, STAGES, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
-          smem, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
+      (void)scale_copy_loop<true, MX, STAGES, NSLOT, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
           abort_flag, limit, 31);
     }
   } else {
@@ -926,16 +924,15 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
     for (int t = cluster_id; t < args.num_tiles; t += num_clusters, ++j) {
       int tm, tn;
       tile_coords(args, t, tm, tn);
-      const uint32_t b = j & 1u;
-      const uint32_t leader_empty = mapa_shared(smem_u32(acc.emp(b, c.wg)), 0);
+      const uint32_t leader_empty = mapa_shared(smem_u32(acc.emp(c.wg)), 0);
       auto release = [&]() {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_empty);
       };
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc.full[b], (j >> 1) & 1u, abort_flag, limit, 27))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(acc.full, j & 1u, abort_flag, limit, 27))) break;
       tc_fence_after();
-      if (!epilogue_tile<EPI>(c, b, tm * 256 + 128 * static_cast<int>(rank), tn * BN, release)) break;
+      if (!epilogue_tile<EPI>(c, tm * 256 + 128 * static_cast<int>(rank), tn * BN, release)) break;
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
