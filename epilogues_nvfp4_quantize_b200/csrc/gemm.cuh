@@ -68,11 +68,19 @@ constexpr int BK_BYTES = BK / 2;        // 128: one swizzle row
 constexpr int SF_UNIT = 512;            // scales of 128 rows x 64 K
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int COPY_WARPS = 2;
-constexpr int NUM_THREADS = EPI_THREADS + 64 + 32 * COPY_WARPS;
+constexpr int COPY_WARPS = 4;
+constexpr int ROLE_WARPS = 8;           // two warpgroups: producer, MMA, copy warps, idle
+constexpr int NUM_THREADS = EPI_THREADS + 32 * ROLE_WARPS;
 constexpr int PRODUCER_WARP = EPI_WARPS;
 constexpr int MMA_WARP = EPI_WARPS + 1;
 constexpr int COPY_WARP0 = EPI_WARPS + 2;
+// Registers per thread after the split: launched with 65536 / 512 = 128 each, the role
+// warpgroups drop to ROLE_REGS and the epilogue warpgroups rise to EPI_REGS.
+constexpr uint32_t EPI_REGS = 184;
+constexpr uint32_t ROLE_REGS = 64;
+constexpr uint32_t LAUNCH_REGS = 65536 / NUM_THREADS;
+static_assert(2 + COPY_WARPS <= ROLE_WARPS, "warp roles");
+static_assert(EPI_THREADS * EPI_REGS + 32 * ROLE_WARPS * ROLE_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr int BOX_BYTES = 32 * 128;     // one staging box: 32 rows x 128 bytes
 constexpr int RED_BYTES = 2 * 2 * 128 * 4;
 constexpr uint32_t TMEM_COLS = 512;
@@ -105,7 +113,7 @@ struct SmemPlan {
   static constexpr int OFF_EPI = S * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_EPI + gemm_cfg::EPI_WARPS * gemm_cfg::BOX_BYTES;
   static constexpr int OFF_BAR = OFF_RED + gemm_cfg::RED_BYTES;
-  static constexpr int NUM_BARS = 3 * S + 7;  // full, empty, 7 more (bar_idx), scales loaded
+  static constexpr int NUM_BARS = 3 * S + 5 + gemm_cfg::COPY_WARPS;  // full, empty, bar_idx, scales loaded
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -129,9 +137,9 @@ constexpr int ACC_EMPTY = 1;  // [2] per epilogue warpgroup: accumulator moved t
 constexpr int RED = 3;
 constexpr int DRAIN = 4;      // MMA warp's own drain on give-up
 constexpr int CP_DRAIN = 5;   // [COPY_WARPS] copy warps' own drain on give-up
-constexpr int SF_LOADED = 7;  // [S] a stage's scale units have landed (their own tx count)
+constexpr int SF_LOADED = CP_DRAIN + gemm_cfg::COPY_WARPS;  // [S] a stage's scale units have landed
 }  // namespace bar_idx
-static_assert(bar_idx::CP_DRAIN + gemm_cfg::COPY_WARPS <= bar_idx::SF_LOADED, "barrier plan");
+static_assert(bar_idx::SF_LOADED == 5 + gemm_cfg::COPY_WARPS, "barrier plan");
 
 // Accumulator hand-off between the MMA warp and the epilogue: one "full" barrier (MMA
 // commit) and one "empty" barrier per warpgroup (one arrival per warp of that warpgroup,
@@ -589,120 +597,124 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   const int ktiles = args.K / BK;
   const int64_t kunits = args.K / ScaleFmt<MX>::K_PER_UNIT;  // scale units per 128-row group along K
 
-  if (warp == EPI_WARPS) {
-    // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
-        int tm, tn;
-        tile_coords(args, t, tm, tn);
-        for (int kt = 0; kt < ktiles; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 1)) {
-            ok = false;
-            break;
+  if (warp >= EPI_WARPS) {
+    regs_release<ROLE_REGS>();
+    if (warp == EPI_WARPS) {
+      // ------------------------------------------------------------------ producer
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
+          int tm, tn;
+          tile_coords(args, t, tm, tn);
+          for (int kt = 0; kt < ktiles; ++kt) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 1)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sb = smem + stage * P::STAGE_BYTES;
+            // scales first, on their own barrier, then the code tiles
+            uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
+            mbar_arrive_expect_tx(sfl, P::SFA_BYTES + P::SFB_BYTES);
+            const int64_t ka = static_cast<int64_t>(kt) * U;
+            uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
+            bulk_load(ssf, args.sfa + (tm * kunits + ka) * SF_UNIT, P::SFA_BYTES, sfl);
+            bulk_load(ssf + P::SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT, P::SFB_BYTES / 2, sfl);
+            bulk_load(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, args.sfb + ((2 * tn + 1) * kunits + ka) * SF_UNIT,
+                      P::SFB_BYTES / 2, sfl);
+            mbar_arrive_expect_tx(&full[stage], P::A_BYTES + P::B_BYTES);
+            tma_load_2d(sb, &tmA, &full[stage], kt * BK_BYTES, tm * BM);
+            tma_load_2d(sb + P::A_BYTES, &tmB, &full[stage], kt * BK_BYTES, tn * BN);
+            ++issued;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          uint8_t* sb = smem + stage * P::STAGE_BYTES;
-          // scales first, on their own barrier, then the code tiles
-          uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
-          mbar_arrive_expect_tx(sfl, P::SFA_BYTES + P::SFB_BYTES);
-          const int64_t ka = static_cast<int64_t>(kt) * U;
-          uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
-          bulk_load(ssf, args.sfa + (tm * kunits + ka) * SF_UNIT, P::SFA_BYTES, sfl);
-          bulk_load(ssf + P::SFA_BYTES, args.sfb + ((2 * tn) * kunits + ka) * SF_UNIT, P::SFB_BYTES / 2, sfl);
-          bulk_load(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, args.sfb + ((2 * tn + 1) * kunits + ka) * SF_UNIT,
-                    P::SFB_BYTES / 2, sfl);
-          mbar_arrive_expect_tx(&full[stage], P::A_BYTES + P::B_BYTES);
-          tma_load_2d(sb, &tmA, &full[stage], kt * BK_BYTES, tm * BM);
-          tma_load_2d(sb + P::A_BYTES, &tmB, &full[stage], kt * BK_BYTES, tn * BN);
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+        }
+        if (ok) {
+          // Tail: wait until the MMAs have released every stage still in use, so that no
+          // arrival reaches this CTA's barriers after it exits.
+          for (int i = 0; i < STAGES && i < issued; ++i) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 13)) break;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        } else {
+          // Give up: wait (bounded) for the copies this thread started, then leave.
+          for (int i = 0; i < STAGES && i < issued; ++i) {
+            if (--stage < 0) {
+              stage = STAGES - 1;
+              phase ^= 1u;
+            }
+            (void)mbar_wait(&full[stage], phase, nullptr, limit, 11);
+            (void)mbar_wait(&xbars[bar_idx::SF_LOADED + stage], phase, nullptr, limit, 11);
           }
         }
       }
-      if (ok) {
-        // Tail: wait until the MMAs have released every stage still in use, so that no
-        // arrival reaches this CTA's barriers after it exits.
-        for (int i = 0; i < STAGES && i < issued; ++i) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 13)) break;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      } else {
-        // Give up: wait (bounded) for the copies this thread started, then leave.
-        for (int i = 0; i < STAGES && i < issued; ++i) {
-          if (--stage < 0) {
-            stage = STAGES - 1;
-            phase ^= 1u;
-          }
-          (void)mbar_wait(&full[stage], phase, nullptr, limit, 11);
-          (void)mbar_wait(&xbars[bar_idx::SF_LOADED + stage], phase, nullptr, limit, 11);
-        }
-      }
-    }
-  } else if (warp == EPI_WARPS + 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = MX ? idesc_mxfp4(BM, BN, 0) : idesc_nvfp4(BM, BN);
-      int stage = 0;
-      uint32_t phase = 0, j = 0;
-      int sl = 0;  // scale slot of this K step
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++j) {
-        if (!acc_acquire(acc, j, abort_flag, limit, 2)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem;
-        for (int kt = 0; kt < ktiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3)) {
+    } else if (warp == EPI_WARPS + 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc = MX ? idesc_mxfp4(BM, BN, 0) : idesc_nvfp4(BM, BN);
+        int stage = 0;
+        uint32_t phase = 0, j = 0;
+        int sl = 0;  // scale slot of this K step
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++j) {
+          if (!acc_acquire(acc, j, abort_flag, limit, 2)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + P::A_BYTES;
-          const uint32_t slot = tmem + sf_slot(sl);
-          const uint64_t adesc = smem_desc_sw128(a_addr);
-          const uint64_t bdesc = smem_desc_sw128(b_addr);
-#pragma unroll
-          for (int kb = 0; kb < BK / 64; ++kb) {
-            // +32 bytes along K per 64 FP4 values: +2 in the descriptor's address field
-            const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
-            const uint32_t id = MX ? (idesc | ((2u * (kb & 1)) << 29) | ((2u * (kb & 1)) << 4)) : idesc;
-            tc_mma_nvfp4<MX>(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, id, slot + 4 * u, slot + SFB_OFF + 8 * u,
-                             (kt > 0 || kb > 0) ? 1u : 0u);
+          const uint32_t d_tmem = tmem;
+          for (int kt = 0; kt < ktiles; ++kt) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, limit, 3)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
+            const uint32_t b_addr = a_addr + P::A_BYTES;
+            const uint32_t slot = tmem + sf_slot(sl);
+            const uint64_t adesc = smem_desc_sw128(a_addr);
+            const uint64_t bdesc = smem_desc_sw128(b_addr);
+  #pragma unroll
+            for (int kb = 0; kb < BK / 64; ++kb) {
+              // +32 bytes along K per 64 FP4 values: +2 in the descriptor's address field
+              const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
+              const uint32_t id = MX ? (idesc | ((2u * (kb & 1)) << 29) | ((2u * (kb & 1)) << 4)) : idesc;
+              tc_mma_nvfp4<MX>(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, id, slot + 4 * u, slot + SFB_OFF + 8 * u,
+                               (kt > 0 || kb > 0) ? 1u : 0u);
+            }
+            tc_commit(&empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            if (++sl == NSLOT) sl = 0;
           }
-          tc_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          if (++sl == NSLOT) sl = 0;
+          if (!ok) break;
+          tc_commit(acc.full);
         }
-        if (!ok) break;
-        tc_commit(acc.full);
+        if (!ok) {
+          tc_commit(drain_bar);
+          (void)mbar_wait(drain_bar, 0, nullptr, limit, 12);
+        }
       }
-      if (!ok) {
-        tc_commit(drain_bar);
-        (void)mbar_wait(drain_bar, 0, nullptr, limit, 12);
+    } else if (warp < COPY_WARP0 + COPY_WARPS) {
+      // ------------------------------------------------------------------ scale copies
+      if (lane == 0) {
+        (void)scale_copy_loop<false, MX, STAGES, NSLOT, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+            smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
+            abort_flag, limit, 14);
       }
-    }
-  } else if (warp >= COPY_WARP0) {
-    // ------------------------------------------------------------------ scale copies
-    if (lane == 0) {
-      (void)scale_copy_loop<false, MX, STAGES, NSLOT, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
-          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, blockIdx.x, gridDim.x),
-          abort_flag, limit, 14);
     }
   } else {
+    regs_acquire<EPI_REGS>();
     // ------------------------------------------------------------------ epilogue
     EpiCtx c = make_epi_ctx(args, &tmD, tmem, smem, P::OFF_EPI, P::OFF_RED, red_bar, abort_flag);
     uint32_t j = 0;
@@ -801,123 +813,127 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
   const int ktiles = args.K / BK;
   const int kunits = args.K / ScaleFmt<MX>::K_PER_UNIT;
 
-  if (warp == EPI_WARPS) {
-    // ------------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters) {
-        int tm, tn;
-        tile_coords(args, t, tm, tn);
-        const int a_row = tm * 256 + 128 * static_cast<int>(rank);   // this CTA's A rows
-        const int b_row = tn * 256 + 128 * static_cast<int>(rank);   // this CTA's half of B
-        const int sfa_group = a_row / 128;
-        for (int kt = 0; kt < ktiles; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 21)) {
-            ok = false;
-            break;
+  if (warp >= EPI_WARPS) {
+    regs_release<ROLE_REGS>();
+    if (warp == EPI_WARPS) {
+      // ------------------------------------------------------------------ producer (both CTAs)
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters) {
+          int tm, tn;
+          tile_coords(args, t, tm, tn);
+          const int a_row = tm * 256 + 128 * static_cast<int>(rank);   // this CTA's A rows
+          const int b_row = tn * 256 + 128 * static_cast<int>(rank);   // this CTA's half of B
+          const int sfa_group = a_row / 128;
+          for (int kt = 0; kt < ktiles; ++kt) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 21)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sb = smem + stage * P::STAGE_BYTES;
+            // both CTAs' bytes count on the leader's barriers: scales first, on their own
+            // barrier, then the code tiles
+            uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
+            const uint32_t bar_sf = mapa_shared(smem_u32(sfl), 0);
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(sfl, 2 * (P::SFA_BYTES + P::SFB_BYTES));
+            // scale units: 512 bytes = 2 rows of the 256-byte-wide scale tensor map
+            uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
+            tma_load_2d_pair(ssf, &tmSFA, bar_sf, 0, 2 * (sfa_group * kunits + U * kt));
+            tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar_sf, 0, 2 * ((2 * tn) * kunits + U * kt));
+            tma_load_2d_pair(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, &tmSFB, bar_sf, 0,
+                             2 * ((2 * tn + 1) * kunits + U * kt));
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (P::A_BYTES + P::B_BYTES));
+            tma_load_2d_pair(sb, &tmA, bar, kt * BK_BYTES, a_row);
+            tma_load_2d_pair(sb + P::A_BYTES, &tmB, bar, kt * BK_BYTES, b_row);
+            ++issued;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          uint8_t* sb = smem + stage * P::STAGE_BYTES;
-          // both CTAs' bytes count on the leader's barriers: scales first, on their own
-          // barrier, then the code tiles
-          uint64_t* sfl = &xbars[bar_idx::SF_LOADED + stage];
-          const uint32_t bar_sf = mapa_shared(smem_u32(sfl), 0);
-          const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(sfl, 2 * (P::SFA_BYTES + P::SFB_BYTES));
-          // scale units: 512 bytes = 2 rows of the 256-byte-wide scale tensor map
-          uint8_t* ssf = sb + P::A_BYTES + P::B_BYTES;
-          tma_load_2d_pair(ssf, &tmSFA, bar_sf, 0, 2 * (sfa_group * kunits + U * kt));
-          tma_load_2d_pair(ssf + P::SFA_BYTES, &tmSFB, bar_sf, 0, 2 * ((2 * tn) * kunits + U * kt));
-          tma_load_2d_pair(ssf + P::SFA_BYTES + P::SFB_BYTES / 2, &tmSFB, bar_sf, 0,
-                           2 * ((2 * tn + 1) * kunits + U * kt));
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (P::A_BYTES + P::B_BYTES));
-          tma_load_2d_pair(sb, &tmA, bar, kt * BK_BYTES, a_row);
-          tma_load_2d_pair(sb + P::A_BYTES, &tmB, bar, kt * BK_BYTES, b_row);
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
+        }
+        if (ok) {
+          for (int i = 0; i < STAGES && i < issued; ++i) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 23)) break;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        } else if (leader) {
+          // both CTAs' copies complete on the leader's barriers: wait (bounded) for them
+          for (int i = 0; i < STAGES && i < issued; ++i) {
+            if (--stage < 0) {
+              stage = STAGES - 1;
+              phase ^= 1u;
+            }
+            (void)mbar_wait(&full[stage], phase, nullptr, limit, 24);
+            (void)mbar_wait(&xbars[bar_idx::SF_LOADED + stage], phase, nullptr, limit, 24);
           }
         }
       }
-      if (ok) {
-        for (int i = 0; i < STAGES && i < issued; ++i) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 23)) break;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      } else if (leader) {
-        // both CTAs' copies complete on the leader's barriers: wait (bounded) for them
-        for (int i = 0; i < STAGES && i < issued; ++i) {
-          if (--stage < 0) {
-            stage = STAGES - 1;
-            phase ^= 1u;
-          }
-          (void)mbar_wait(&full[stage], phase, nullptr, limit, 24);
-          (void)mbar_wait(&xbars[bar_idx::SF_LOADED + stage], phase, nullptr, limit, 24);
-        }
-      }
-    }
-  } else if (warp == EPI_WARPS + 1) {
-    // ------------------------------------------------------------------ MMA issuer (leader only)
-    if (leader && lane == 0) {
-      const uint32_t idesc = MX ? idesc_mxfp4(2 * BM, BN, 0) : idesc_nvfp4(2 * BM, BN);
-      int stage = 0;
-      uint32_t phase = 0, j = 0;
-      int sl = 0;  // scale slot of this K step
-      bool ok = true;
-      for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters, ++j) {
-        if (!acc_acquire(acc, j, abort_flag, limit, 22)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem;
-        for (int kt = 0; kt < ktiles; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25)) {
+    } else if (warp == EPI_WARPS + 1) {
+      // ------------------------------------------------------------------ MMA issuer (leader only)
+      if (leader && lane == 0) {
+        const uint32_t idesc = MX ? idesc_mxfp4(2 * BM, BN, 0) : idesc_nvfp4(2 * BM, BN);
+        int stage = 0;
+        uint32_t phase = 0, j = 0;
+        int sl = 0;  // scale slot of this K step
+        bool ok = true;
+        for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters, ++j) {
+          if (!acc_acquire(acc, j, abort_flag, limit, 22)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + P::A_BYTES;
-          const uint32_t slot = tmem + sf_slot(sl);
-          const uint64_t adesc = smem_desc_sw128(a_addr);
-          const uint64_t bdesc = smem_desc_sw128(b_addr);
-#pragma unroll
-          for (int kb = 0; kb < BK / 64; ++kb) {
-            const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
-            const uint32_t id = MX ? (idesc | ((2u * (kb & 1)) << 29) | ((2u * (kb & 1)) << 4)) : idesc;
-            tc_mma_nvfp4_pair<MX>(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, id, slot + 4 * u, slot + SFB_OFF + 8 * u,
-                                  (kt > 0 || kb > 0) ? 1u : 0u);
+          const uint32_t d_tmem = tmem;
+          for (int kt = 0; kt < ktiles; ++kt) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, limit, 25)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
+            const uint32_t b_addr = a_addr + P::A_BYTES;
+            const uint32_t slot = tmem + sf_slot(sl);
+            const uint64_t adesc = smem_desc_sw128(a_addr);
+            const uint64_t bdesc = smem_desc_sw128(b_addr);
+  #pragma unroll
+            for (int kb = 0; kb < BK / 64; ++kb) {
+              const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
+              const uint32_t id = MX ? (idesc | ((2u * (kb & 1)) << 29) | ((2u * (kb & 1)) << 4)) : idesc;
+              tc_mma_nvfp4_pair<MX>(d_tmem, adesc + 2 * kb, bdesc + 2 * kb, id, slot + 4 * u, slot + SFB_OFF + 8 * u,
+                                    (kt > 0 || kb > 0) ? 1u : 0u);
+            }
+            tc_commit_pair(&empty[stage], 0x3);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            if (++sl == NSLOT) sl = 0;
           }
-          tc_commit_pair(&empty[stage], 0x3);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-          if (++sl == NSLOT) sl = 0;
+          if (!ok) break;
+          tc_commit_pair(acc.full, 0x3);
         }
-        if (!ok) break;
-        tc_commit_pair(acc.full, 0x3);
+        if (!ok) {
+          tc_commit_pair(drain_bar, 0x1);
+          (void)mbar_wait(drain_bar, 0, nullptr, limit, 26);
+        }
       }
-      if (!ok) {
-        tc_commit_pair(drain_bar, 0x1);
-        (void)mbar_wait(drain_bar, 0, nullptr, limit, 26);
+    } else if (warp < COPY_WARP0 + COPY_WARPS) {
+      // ------------------------------------------------------------------ scale copies (leader only)
+      if (leader && lane == 0) {
+        (void)scale_copy_loop<true, MX, STAGES, NSLOT, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
+            smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
+            abort_flag, limit, 31);
       }
-    }
-  } else if (warp >= COPY_WARP0) {
-    // ------------------------------------------------------------------ scale copies (leader only)
-    if (leader && lane == 0) {
-      (void)scale_copy_loop<true, MX, STAGES, NSLOT, P::STAGE_BYTES, P::A_BYTES + P::B_BYTES, P::SFB_BYTES / 2>(
-          smem, full, xbars, tmem, warp - COPY_WARP0, ksteps_of(args.num_tiles, args.K, cluster_id, num_clusters),
-          abort_flag, limit, 31);
     }
   } else {
+    regs_acquire<EPI_REGS>();
     // ------------------------------------------------------------------ epilogue (both CTAs)
     EpiCtx c = make_epi_ctx(args, &tmD, tmem, smem, P::OFF_EPI, P::OFF_RED, red_bar, abort_flag);
     uint32_t j = 0;

@@ -67,6 +67,20 @@ nvfp4_status launch_status() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The GEMM kernels split their registers between warpgroups at run time (setmaxnreg): the
+// epilogue warpgroups can only grow if the block was launched with enough registers for
+// the whole split, otherwise they would wait forever. Checked once per kernel, before its
+// first launch.
+template <class Kernel>
+bool register_split_fits(Kernel kern) {
+  using namespace nvfp4::gemm_cfg;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+  const long long launched = static_cast<long long>(fa.numRegs) * NUM_THREADS;
+  const long long needed = static_cast<long long>(EPI_THREADS) * EPI_REGS + 32ll * ROLE_WARPS * ROLE_REGS;
+  return launched >= needed;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -172,6 +186,7 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
     {
       std::lock_guard<std::mutex> lock(g_mutex);
       if (!info->gemm_attr_set[EPI + 4 * MX]) {
+        if (!register_split_fits(kern)) return NVFP4_ERR_CUDA;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
           return NVFP4_ERR_CUDA;
         info->gemm_attr_set[EPI + 4 * MX] = true;
@@ -201,6 +216,7 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!info->pair_attr_set[EPI + 4 * MX]) {
+      if (!register_split_fits(kern)) return NVFP4_ERR_CUDA;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
         return NVFP4_ERR_CUDA;
       cfg.gridDim = dim3(2 * (info->sm_count / 2), 1, 1);
