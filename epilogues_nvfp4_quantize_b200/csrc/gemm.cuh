@@ -645,7 +645,9 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             }
           }
         } else {
-          // Give up: wait (bounded) for the copies this thread started, then leave.
+          // Give up: wait (bounded) for the copies this thread started, then leave. The operand
+          // barrier also counts the copy warps' commits; a stage whose scale copies were never
+          // made keeps it open, and that wait then ends at its limit.
           for (int i = 0; i < STAGES && i < issued; ++i) {
             if (--stage < 0) {
               stage = STAGES - 1;
@@ -664,6 +666,14 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
         uint32_t phase = 0, j = 0;
         int sl = 0;  // scale slot of this K step
         bool ok = true;
+        // operand descriptors and scale slot advance with the ring instead of being rebuilt
+        // from the stage index: fewer instructions in the thread that paces the tensor pipe
+        const uint64_t adesc0 = smem_desc_sw128(smem_u32(smem));
+        constexpr uint64_t STAGE_DESC = P::STAGE_BYTES >> 4;  // the descriptor's address unit is 16 B
+        constexpr uint64_t B_DESC = P::A_BYTES >> 4;
+        static_assert((STAGES * P::STAGE_BYTES) >> 4 < (1 << 14), "descriptor address field");
+        uint64_t adesc = adesc0;
+        uint32_t slot = tmem + sf_slot(0);
         for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++j) {
           if (!acc_acquire(acc, j, abort_flag, limit, 2)) {
             ok = false;
@@ -677,11 +687,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
-            const uint32_t b_addr = a_addr + P::A_BYTES;
-            const uint32_t slot = tmem + sf_slot(sl);
-            const uint64_t adesc = smem_desc_sw128(a_addr);
-            const uint64_t bdesc = smem_desc_sw128(b_addr);
+            const uint64_t bdesc = adesc + B_DESC;
   #pragma unroll
             for (int kb = 0; kb < BK / 64; ++kb) {
               // +32 bytes along K per 64 FP4 values: +2 in the descriptor's address field
@@ -691,11 +697,17 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
                                (kt > 0 || kb > 0) ? 1u : 0u);
             }
             tc_commit(&empty[stage]);
+            adesc += STAGE_DESC;
+            slot += SF_SLOT_COLS;
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
+              adesc = adesc0;
             }
-            if (++sl == NSLOT) sl = 0;
+            if (++sl == NSLOT) {
+              sl = 0;
+              slot = tmem + sf_slot(0);
+            }
           }
           if (!ok) break;
           tc_commit(acc.full);
@@ -865,7 +877,9 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
             }
           }
         } else if (leader) {
-          // both CTAs' copies complete on the leader's barriers: wait (bounded) for them
+          // both CTAs' copies complete on the leader's barriers: wait (bounded) for them. The
+          // operand barrier also counts the copy warps' commits; a stage whose copies were never
+          // made keeps it open, and that wait then ends at its limit.
           for (int i = 0; i < STAGES && i < issued; ++i) {
             if (--stage < 0) {
               stage = STAGES - 1;
@@ -884,6 +898,14 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
         uint32_t phase = 0, j = 0;
         int sl = 0;  // scale slot of this K step
         bool ok = true;
+        // operand descriptors and scale slot advance with the ring instead of being rebuilt
+        // from the stage index: fewer instructions in the thread that paces the tensor pipe
+        const uint64_t adesc0 = smem_desc_sw128(smem_u32(smem));
+        constexpr uint64_t STAGE_DESC = P::STAGE_BYTES >> 4;  // the descriptor's address unit is 16 B
+        constexpr uint64_t B_DESC = P::A_BYTES >> 4;
+        static_assert((STAGES * P::STAGE_BYTES) >> 4 < (1 << 14), "descriptor address field");
+        uint64_t adesc = adesc0;
+        uint32_t slot = tmem + sf_slot(0);
         for (int t = cluster_id; ok && t < args.num_tiles; t += num_clusters, ++j) {
           if (!acc_acquire(acc, j, abort_flag, limit, 22)) {
             ok = false;
@@ -897,11 +919,7 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + stage * P::STAGE_BYTES);
-            const uint32_t b_addr = a_addr + P::A_BYTES;
-            const uint32_t slot = tmem + sf_slot(sl);
-            const uint64_t adesc = smem_desc_sw128(a_addr);
-            const uint64_t bdesc = smem_desc_sw128(b_addr);
+            const uint64_t bdesc = adesc + B_DESC;
   #pragma unroll
             for (int kb = 0; kb < BK / 64; ++kb) {
               const int u = MX ? kb >> 1 : kb;  // scale unit of this MMA
@@ -910,11 +928,17 @@ __global__ void __launch_bounds__(gemm_cfg::NUM_THREADS, 1)
                                     (kt > 0 || kb > 0) ? 1u : 0u);
             }
             tc_commit_pair(&empty[stage], 0x3);
+            adesc += STAGE_DESC;
+            slot += SF_SLOT_COLS;
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
+              adesc = adesc0;
             }
-            if (++sl == NSLOT) sl = 0;
+            if (++sl == NSLOT) {
+              sl = 0;
+              slot = tmem + sf_slot(0);
+            }
           }
           if (!ok) break;
           tc_commit_pair(acc.full, 0x3);

@@ -182,6 +182,14 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
   const int64_t per_rs = (num_g + NB - 1) / NB;             // chunks per R-row slab
   const int64_t chunks = ((rows_pad + R - 1) / R) * per_rs;
   const int passes = a.compute_amax ? 2 : 1;
+  // This CTA's chunks are blockIdx.x + k * gridDim.x, k < my_chunks. The quantise pass after an
+  // amax pass walks them backwards: the chunks read last by the amax pass are the likeliest
+  // to still be in L2.
+  const int64_t my_chunks = blockIdx.x < chunks ? (chunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto chunk_of = [&](int pass, int64_t k) -> int64_t {
+    const int64_t kk = pass == 1 ? my_chunks - 1 - k : k;
+    return static_cast<int64_t>(blockIdx.x) + kk * gridDim.x;
+  };
 
   if (warp == CONSUMER_WARPS) {
     // ---------------------------------------------------------------- TMA producer
@@ -194,7 +202,8 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
       bool ok = true;
       for (int pass = 0; ok && pass < passes; ++pass) {
         const uint64_t pol = pass + 1 < passes ? keep : stream;
-        for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
+        for (int64_t k = 0; k < my_chunks; ++k) {
+          const int64_t c = chunk_of(pass, k);
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 41)) {
             ok = false;
             break;
@@ -281,7 +290,8 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
       }
       enc = scale_encode_factor(G);
     }
-    for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
+    for (int64_t k = 0; k < my_chunks; ++k) {
+      const int64_t c = chunk_of(pass, k);
       if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, limit, 45))) return;
       const int64_t rs = c / per_rs;
       const int64_t g = (c - rs * per_rs) * NB + b;
