@@ -53,7 +53,7 @@ def workload_desc(M: int) -> str:
 # capture summarised in profiles/, keyed by a hash of the GEMM's device sources: a value
 # taken on another version of the kernel is not reported.
 TRAFFIC_BY_SOURCE = {
-    "562ab63819fb15bb": 146.4e6,
+    "ed135143128cf7a3": 146.4e6,
 }
 
 
@@ -445,7 +445,7 @@ def run_cuda(args):
             "static_gbs": round(fq_bytes / (t_fq_static * 1e-3) / 1e9, 1),
             "hbm_peak_gbs": pk["hbm_gbs"],
             "note": "algorithmic bytes = 2 B read + 2 B written per element; with amax the kernel "
-                    "reads x twice (the second time mostly from L2)",
+                    "reads x twice",
         }
         del y_fq
 
@@ -694,6 +694,145 @@ def run_sweep(args):
         raise SystemExit(f"device status {status}")
 
 
+# ----------------------------------------------------------------------------------
+# the named configurations: fused vs unfused, each timed alone
+# ----------------------------------------------------------------------------------
+def run_configs(args):
+    """The five named problems (the tiny QK-norm case, SwiGLU at M=1024, the 1K-image QKV
+    block, the 1K-image FFN block's up GEMM with re-quantisation and its down GEMM), each
+    timed alone like the sweep: cold L2 (a 512 MB buffer written before each run), 10
+    warm-ups, median of --sweep-runs runs, fused against the plain GEMM plus separate op
+    kernels. cpu_baseline per problem: the oracle on a row sample (all rows of the tiny
+    case), with B's packing done before timing, extrapolated linearly in M."""
+    import torch
+    import epilogues_nvfp4_quantize_b200 as ep
+    import workloads as wk
+    from oracle import nvfp4_oracle as o
+    from epilogues_nvfp4_quantize_b200.build import build
+
+    build()
+    ep.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T = ep.NVFP4Tensor
+    scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    pk = peaks()
+    fp4_peak = pk["bf16"] * FP4_PER_BF16
+    cores = _blas_threads()
+
+    def median_us(fn, runs):
+        for _ in range(10):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(runs)]
+        for e0, e1 in evs:
+            scrub.fill_(1)
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize(dev)
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
+
+    def oracle_s(wl, a, b, w=None, sample=256):
+        rows = None if wl.M <= sample else np.sort(np.random.default_rng(0).choice(wl.M, size=sample,
+                                                                                    replace=False))
+        bq = o.quantized_operand(b)  # weight packing, once per model: not timed
+        t0 = time.perf_counter()
+        if wl.op == "rmsnorm":
+            o.problem_rmsnorm(a, b, w, wl.head_dim, wl.n_norm_cols, wl.eps, rows=rows, b_quant=bq)
+        elif wl.op == "swiglu":
+            ref = o.problem_swiglu(a, b, rows=rows, b_quant=bq)
+            if wl.requant:
+                o.requantize(ref, np.float32(np.abs(ref).max() / 2688))
+        else:
+            o.problem_plain(a, b, rows=rows, b_quant=bq)
+        t = time.perf_counter() - t0
+        n = wl.M if rows is None else len(rows)
+        return t * wl.M / n, n
+
+    n_launch0 = ep.launch_count()
+    down_a = None
+    for name, wl in (("1", wk.qk_norm_tiny()), ("2", wk.swiglu_1024()), ("3", wk.qkv(4096, 256)),
+                     ("4a", wk.ffn_up(4096, True)), ("4b", wk.ffn_down(4096))):
+        inp = wk.make_inputs(wl)
+        a_cpu, b_cpu = inp["a"], inp["b"]
+        a, b = a_cpu.to(dev), b_cpu.to(dev)
+        M, K, N = wl.M, wl.K, wl.N
+        A = T.empty(M, K, dev)
+        ep.nvfp4_quantize(a, A)
+        w_cpu = None
+        if wl.op == "rmsnorm":
+            B = T.empty(N, K, dev)
+            ep.nvfp4_quantize(b, B)
+            w_cpu = inp["w"]
+            w = torch.from_numpy(w_cpu).to(dev)
+            D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+            def fused():
+                ep.gemm_nvfp4_rmsnorm(A, B, w, wl.head_dim, wl.n_norm_cols, wl.eps, D)
+
+            def unfused():
+                ep.gemm_nvfp4_plain(A, B, D)
+                ep.rmsnorm_heads_bf16(D, w, wl.head_dim, wl.n_norm_cols, wl.eps, D)
+        elif wl.op == "swiglu":
+            nh = N // 2
+            Bi, Bl = T.empty(N, K, dev), T.empty(N, K, dev)
+            ep.nvfp4_quantize(b, Bi, interleave=True)
+            ep.nvfp4_quantize(b, Bl)
+            C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            Y = torch.empty(M, nh, dtype=torch.bfloat16, device=dev)
+            if wl.requant:
+                Dq = T.empty(M, nh, dev)
+                ep.gemm_nvfp4_swiglu(A, Bi, Y, None)
+                ep.nvfp4_quantize(Y, Dq)  # static scale of the re-quantised output, calibrated once
+                Dq2 = T(torch.empty_like(Dq.codes), torch.empty_like(Dq.sf), Dq.gscale, M, nh)
+                down_a = Dq  # the down GEMM's A, as in the FFN block
+
+                def fused():
+                    ep.gemm_nvfp4_swiglu(A, Bi, None, Dq)
+
+                def unfused():
+                    ep.gemm_nvfp4_plain(A, Bl, C)
+                    ep.swiglu_bf16(C, Y)
+                    ep.nvfp4_quantize(Y, Dq2, compute_amax=False)
+            else:
+                D = torch.empty(M, nh, dtype=torch.bfloat16, device=dev)
+
+                def fused():
+                    ep.gemm_nvfp4_swiglu(A, Bi, D, None)
+
+                def unfused():
+                    ep.gemm_nvfp4_plain(A, Bl, C)
+                    ep.swiglu_bf16(C, Y)
+        else:
+            B = T.empty(N, K, dev)
+            ep.nvfp4_quantize(b, B)
+            Ad = down_a if down_a is not None else A
+            D = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+            def fused():
+                ep.gemm_nvfp4_plain(Ad, B, D)
+
+            unfused = None  # a plain GEMM has no op to split off
+        tf = median_us(fused, args.sweep_runs)
+        tu = median_us(unfused, args.sweep_runs) if unfused is not None else None
+        t_cpu, n_rows = oracle_s(wl, a_cpu, b_cpu, w_cpu)
+        r = {"config": name, "workload": wl.name, "gflop": round(wl.flops / 1e9, 2), "fused_us": round(tf, 2),
+             "fused_tflops": round(wl.flops / (tf * 1e-6) / 1e12, 1),
+             "pct_fp4_peak": round(100.0 * wl.flops / (tf * 1e-6) / 1e12 / fp4_peak, 1),
+             "unfused_us": None if tu is None else round(tu, 2),
+             "speedup": None if tu is None else round(tu / tf, 3),
+             "cpu_baseline": {"seconds": round(t_cpu, 2), "cores": cores, "kind": "oracle",
+                              "sample": "all rows" if n_rows == M else f"{n_rows} rows, scaled to M={M}"}}
+        print(json.dumps(r), flush=True)
+        torch.cuda.empty_cache()
+    status = ep.read_device_status()
+    print(json.dumps({"configs": "fused vs unfused, cold L2", "runs": args.sweep_runs, "warmup": 10,
+                      "fp4_peak_tflops": round(fp4_peak, 1), "peak_source": pk["source"],
+                      "launches": ep.launch_count() - n_launch0, "device_status": status}), flush=True)
+    if status != 0:
+        raise SystemExit(f"device status {status}")
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -740,6 +879,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="fused vs unfused over M in {1024, 4096, 8192, 16384} x {QKV hd128, hd256, FFN-up}")
     ap.add_argument("--sweep-runs", type=int, default=50)
+    ap.add_argument("--configs", action="store_true",
+                    help="time the five named problems fused vs unfused (cold L2), with the oracle's time")
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -750,6 +891,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.configs:
+        run_configs(args)
     else:
         run_cuda(args)
 
