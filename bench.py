@@ -50,20 +50,27 @@ def workload_desc(M: int) -> str:
 
 
 # DRAM bytes (read + write) per launch of the FFN-up fused GEMM at M=16384, from the ncu
-# capture summarised in profiles/, keyed by a hash of the GEMM's device sources: a value
+# capture summarised in profiles/, keyed by a hash of the GEMM's device code: a value
 # taken on another version of the kernel is not reported.
 TRAFFIC_BY_SOURCE = {
-    "ed135143128cf7a3": 146.4e6,
+    "994dbafb418259f6": 146.4e6,
 }
 
 
 def gemm_source_hash() -> str:
+    """Hash of the GEMM's device sources with comments and blank space removed: the
+    counters depend on the code, so a comment edit keeps the recorded traffic valid. (These
+    sources hold no '//' inside string literals.)"""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "epilogues_nvfp4_quantize_b200", "csrc")
     for f in ("gemm.cuh", "ptx.cuh", "codec.cuh", "unfused.cuh"):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

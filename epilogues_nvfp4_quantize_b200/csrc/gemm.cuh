@@ -10,9 +10,10 @@
 //       stages its own 128 rows of A and 128 of the 256 rows of B, so a CTA moves
 //       38 KB per K step of 256 for 128 x 256 x 256 MMA work (5-stage ring);
 //   gemm_nvfp4_kernel       (M % 256 == 128) one CTA per 128 x 256 tile (3-stage ring).
-// Warp roles (384 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
-// and MMA issuer, warps 10-11 copy the block scales from shared memory into TMEM
-// (tcgen05.cp).
+// Warp roles (512 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
+// and MMA issuer, warps 10-13 copy the block scales from shared memory into TMEM
+// (tcgen05.cp), warps 14-15 idle. The role warpgroups run on 64 registers a thread and the
+// epilogue warpgroups on 184 (setmaxnreg).
 // Issue cost sets the main loop's pace. A tcgen05.mma holds up its issuing thread for
 // about as long as the tensor pipe takes to run it (M 256 x N 256 x K 64: 128 cycles),
 // so the pipe holds no backlog. Whatever else that thread does between two K steps leaves
