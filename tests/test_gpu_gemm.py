@@ -42,6 +42,28 @@ def test_plain_gemm_is_exact_on_exactly_representable_inputs(M, N, K):
     assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} outputs differ"
 
 
+@pytest.mark.parametrize("M", [8192, 8064])
+def test_plain_gemm_exact_over_many_ring_wraps(M):
+    """Many K steps per CTA (or CTA pair), about 35, through the 5-stage ring with 4 TMEM
+    scale slots (CTA pair, M = 8192) and the 3-stage ring with 3 slots (single CTA, M = 8064).
+    The stage and slot counters wrap against each other and across tile boundaries (4 K steps
+    per tile). Exactly representable inputs make every output bit-exact; rows are sampled,
+    always including the first and the last."""
+    N, K = 5120, 1024
+    qa, sa, qb, sb = _exact_operands(M, N, K, seed=77)
+    A = nvfp4_from_arrays(qa, sa, 1.0)
+    B = nvfp4_from_arrays(qb, sb, 1.0)
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_plain(A, B, D)
+    rng = np.random.default_rng(M)
+    rows = np.sort(np.concatenate([[0, M - 1], rng.choice(np.arange(1, M - 1), size=254, replace=False)]))
+    ref = o.bf16_round(o.gemm(o.dequantize(qa[rows], sa[rows], 1.0), o.dequantize(qb, sb, 1.0)))
+    got = bf16_bits(D[torch.from_numpy(rows).to(device())])
+    want = o.bf16_bits(ref)
+    assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} outputs differ"
+    assert ep.read_device_status() == 0
+
+
 def test_plain_gemm_scales_by_both_global_scales():
     M, N, K = 128, 256, 512
     qa, sa, qb, sb = _exact_operands(M, N, K, seed=5)
