@@ -357,6 +357,21 @@ def run_cuda(args):
         t_fused_up = time_loop(lambda: ep.gemm_nvfp4_swiglu(layer.xq, layer.Wup, None, layer.h), args.cmp_steps, 3,
                                torch)
         t_unf_up = time_loop(layer.unfused_up, args.cmp_steps, 3, torch)
+        # the unfused path's op kernels alone, with the HBM bytes each must move
+        t_rms = time_loop(lambda: ep.rmsnorm_heads_bf16(layer.qkv, layer.w_norm, HD, N_NORM, EPS, layer.qkv),
+                          args.cmp_steps, 3, torch)
+        t_swi = time_loop(lambda: ep.swiglu_bf16(layer.c_up, layer.y_up), args.cmp_steps, 3, torch)
+        t_rq = time_loop(lambda: ep.nvfp4_quantize(layer.y_up, layer.h2, compute_amax=False), args.cmp_steps, 3,
+                         torch)
+        b_rms = M * N_NORM * 2 * 2                           # read + write the normalised bf16 columns
+        b_swi = M * N_UP * 2 + M * (N_UP // 2) * 2           # read gate|up, write the product
+        b_rq = M * (N_UP // 2) * (2 + 0.5 + 1 / 16)         # read bf16, write codes + scales
+        op_kernels = {
+            "rmsnorm_heads_bf16": {"us": round(t_rms * 1e3, 1), "gbs": round(b_rms / (t_rms * 1e-3) / 1e9, 1)},
+            "swiglu_bf16": {"us": round(t_swi * 1e3, 1), "gbs": round(b_swi / (t_swi * 1e-3) / 1e9, 1)},
+            "nvfp4_quantize_static": {"us": round(t_rq * 1e3, 1), "gbs": round(b_rq / (t_rq * 1e-3) / 1e9, 1)},
+            "hbm_peak_gbs": pk["hbm_gbs"],
+        }
         result["unfused"] = {
             "qkv": {"fused_us": t_fused_qkv * 1e3, "unfused_us": t_unf_qkv * 1e3,
                     "speedup": t_unf_qkv / t_fused_qkv},
@@ -364,6 +379,7 @@ def run_cuda(args):
                        "speedup": t_unf_up / t_fused_up},
             "note": "unfused = plain NVFP4 GEMM writing bf16, then rmsnorm_heads_bf16 (in place) / "
                     "swiglu_bf16 + nvfp4_quantize (static scale); same kernels' library",
+            "op_kernels": op_kernels,
         }
         del layer.c_up, layer.y_up
         torch.cuda.empty_cache()

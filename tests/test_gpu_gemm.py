@@ -198,6 +198,13 @@ def test_unfused_ops_match_oracle():
         ep.rmsnorm_heads_bf16(xd, torch.from_numpy(w2).to(device()), hd2, N, 1e-6, y2)
         ref2 = o.bf16_round(o.rmsnorm_heads(x.double().numpy(), w2, hd2, N, 1e-6))
         assert_close(bf16_to_np(y2), ref2, "rmsnorm_heads_bf16 hd128")
+    # a head count that is not a multiple of the kernel's heads per warp, computed in place
+    xr = wk.activations(7, 768, 0, seed=11)
+    wr = np.tile(wk.norm_weight(hd, 11), 3).astype(np.float32)
+    yr = xr.to(device())
+    ep.rmsnorm_heads_bf16(yr, torch.from_numpy(wr).to(device()), hd, 768, 1e-6, yr)
+    refr = o.bf16_round(o.rmsnorm_heads(xr.double().numpy(), wr, hd, 768, 1e-6))
+    assert_close(bf16_to_np(yr), refr, "rmsnorm_heads_bf16 ragged, in place")
     c = wk.activations(M, 2 * 512, 0, seed=10).to(device())
     ys = torch.empty(M, 512, dtype=torch.bfloat16, device=device())
     ep.swiglu_bf16(c, ys)
