@@ -16,8 +16,8 @@
 // epilogue warpgroups on 184 (setmaxnreg).
 // Issue cost sets the main loop's pace. A tcgen05.mma holds up its issuing thread for
 // about as long as the tensor pipe takes to run it (M 256 x N 256 x K 64: 128 cycles),
-// so the pipe holds no backlog. Whatever else that thread does between two K steps leaves
-// the pipe idle. So the MMA thread does only this per K step: one wait on the stage's
+// so the pipe holds about one MMA of backlog at most. Whatever else that thread does
+// between two K steps beyond that leaves the pipe idle. So the MMA thread does only this per K step: one wait on the stage's
 // barrier, the 4 MMAs and one commit that frees the stage.
 // - The scale copies are issued from their own warps, on other SM sub-partitions.
 // - The copy warps' commits land on the same stage barrier as the operand bytes, so one
