@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     gemm_mxfp4_swiglu,
     gemm_nvfp4_plain,
     gemm_nvfp4_pointwise,
+    gemm_nvfp4_reduce_rows_f32,
     gemm_nvfp4_rmsnorm,
     gemm_nvfp4_swiglu,
     launch_count,

@@ -26,7 +26,7 @@ EXPORTS = (
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
     "nvfp4_quantize_noalloc", "nvfp4_fake_quantize", "gemm_nvfp4_pointwise",
     "mxfp4_sf_bytes", "mxfp4_quantize", "gemm_mxfp4_pointwise", "gemm_mxfp4_plain",
-    "gemm_mxfp4_rmsnorm", "gemm_mxfp4_swiglu",
+    "gemm_mxfp4_rmsnorm", "gemm_mxfp4_swiglu", "gemm_nvfp4_reduce_rows_f32",
 )
 
 
@@ -63,6 +63,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_quantize_noalloc": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
         "nvfp4_fake_quantize": (i32, [vp, i64, i64, i64, i32, vp, vp, i64, vp, vp]),
         "gemm_nvfp4_pointwise": (i32, [_Tensor, _Tensor, vp, i32, i32, vp, i64, ctypes.POINTER(_Tensor), vp]),
+        "gemm_nvfp4_reduce_rows_f32": (i32, [_Tensor, _Tensor, vp, i32, i64, i64, vp]),
         "mxfp4_sf_bytes": (i64, [i64, i64]),
         "mxfp4_quantize": (i32, [vp, i64, i64, i64, i32, _Tensor, vp]),
         "gemm_mxfp4_pointwise": (i32, [_Tensor, _Tensor, vp, i32, i32, vp, i64, vp]),
@@ -194,6 +195,17 @@ def gemm_nvfp4_pointwise(A: NVFP4Tensor, B: NVFP4Tensor, D: Optional[torch.Tenso
     _check(load().gemm_nvfp4_pointwise(A.c(), B.c(), _ptr(bias), ACT_RELU if relu else ACT_NONE, kind, p, ld, dq,
                                        _stream(stream)), "gemm_nvfp4_pointwise")
     return D, Dq
+
+
+def gemm_nvfp4_reduce_rows_f32(A: NVFP4Tensor, B: NVFP4Tensor, dst_ptrs: torch.Tensor, rows_per_rank: int,
+                               ldd: int, stream=None):
+    """Add row m of G_A G_B (A B^T) (float32) into destination m // rows_per_rank at row
+    m % rows_per_rank (see gemm_nvfp4_reduce_rows_f32 in the header). dst_ptrs: a device
+    int64 tensor of the destinations' addresses (float32 blocks with leading dimension ldd)."""
+    if dst_ptrs.dtype != torch.int64 or dst_ptrs.dim() != 1 or not dst_ptrs.is_cuda or not dst_ptrs.is_contiguous():
+        raise ValueError("dst_ptrs must be a contiguous 1-D int64 tensor on the GPU")
+    _check(load().gemm_nvfp4_reduce_rows_f32(A.c(), B.c(), dst_ptrs.data_ptr(), dst_ptrs.numel(), rows_per_rank, ldd,
+                                             _stream(stream)), "gemm_nvfp4_reduce_rows_f32")
 
 
 MXFP4_HADAMARD32 = 2

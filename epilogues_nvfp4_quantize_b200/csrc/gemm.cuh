@@ -58,7 +58,7 @@
 
 namespace nvfp4 {
 
-enum EpiKind { EPI_PLAIN = 0, EPI_RMSNORM = 1, EPI_SWIGLU = 2, EPI_POINTWISE = 3 };
+enum EpiKind { EPI_PLAIN = 0, EPI_RMSNORM = 1, EPI_SWIGLU = 2, EPI_POINTWISE = 3, EPI_REDUCE = 4 };
 enum OutKind { OUT_BF16 = 0, OUT_F16 = 1, OUT_F32 = 2 };
 
 namespace gemm_cfg {
@@ -270,6 +270,11 @@ struct GemmArgs {
   uint8_t* q_sf;
   const float* q_gscale;
   int q_cols;           // its columns (Nh, or N)
+  // row-parallel reduction (EPI_REDUCE): row m of alpha * acc is added into
+  // red_dst[m / red_rows] + (m % red_rows) * red_ldd
+  float* const* red_dst;
+  int64_t red_rows;
+  int64_t red_ldd;
   uint64_t wait_limit_ns;
 };
 
@@ -302,6 +307,20 @@ __device__ __forceinline__ void flush_box(const CUtensorMap* map, uint8_t* box, 
     tma_store_2d(map, box, x, y);
     bulk_commit();
   }
+}
+
+// Add this warp's staging box (32 rows x 32 floats, 128-byte swizzle) into dst (row pitch ldd
+// floats): each instruction adds 4 whole 128-byte rows, 8 lanes per row, 16 bytes a lane.
+__device__ __forceinline__ void red_box_f32(const uint8_t* box, int lane, float* dst, int64_t ldd) {
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int idx = it * 32 + lane;
+    const int row = idx >> 3, q = idx & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(box + row * 128 + ((q ^ (row & 7)) << 4));
+    red_add_v4_f32(dst + static_cast<int64_t>(row) * ldd + 4 * q, v);
+  }
+  __syncwarp();
 }
 
 __device__ __forceinline__ void box_reuse_wait(int lane) {
@@ -382,6 +401,20 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
       dst[0] = make_uint4(qc[0], qc[1], qc[2], qc[3]);
       dst[1] = make_uint4(qc[4], qc[5], qc[6], qc[7]);
       *reinterpret_cast<uint32_t*>(args.q_sf + sf_word_offset(row, oc0 >> 4, args.q_cols >> 4)) = sfw;
+    }
+    return true;
+  } else if constexpr (EPI == EPI_REDUCE) {
+    // Row-parallel GEMM with its reduce-scatter fused in: this warp's 32 rows all belong to
+    // one destination (red_rows is a multiple of 128), into which alpha * acc is added.
+    const int64_t row0 = m0 + c.sub * 32;
+    const int64_t owner = row0 / args.red_rows;
+    float* dst = args.red_dst[owner] + (row0 - owner * args.red_rows) * args.red_ldd + col0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[q][j] = __float_as_uint(__fmul_rn(alpha, __uint_as_float(v[q][j])));
+      stage_row_bf16(c.box, lane, v[q]);  // 32 words: 32 floats of the row
+      red_box_f32(c.box, lane, dst + 32 * q, args.red_ldd);
     }
     return true;
   } else if constexpr (EPI == EPI_POINTWISE) {

@@ -25,15 +25,16 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr int kMaxDevices = 64;
 
 std::atomic<int64_t> g_launches{0};
+constexpr int kEpiKinds = nvfp4::EPI_REDUCE + 1;
 
 struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sm_count = 0;
-  // per kernel instance: index epilogue kind + 4 * (MXFP4 scales)
-  bool gemm_attr_set[8] = {};
-  bool pair_attr_set[8] = {};
-  int pair_clusters[8] = {};
+  // per kernel instance: index epilogue kind + kEpiKinds * (MXFP4 scales)
+  bool gemm_attr_set[2 * kEpiKinds] = {};
+  bool pair_attr_set[2 * kEpiKinds] = {};
+  int pair_clusters[2 * kEpiKinds] = {};
   bool quant_attr_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -185,11 +186,11 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
     auto kern = nvfp4::gemm_nvfp4_kernel<EPI, MX>;
     {
       std::lock_guard<std::mutex> lock(g_mutex);
-      if (!info->gemm_attr_set[EPI + 4 * MX]) {
+      if (!info->gemm_attr_set[EPI + kEpiKinds * MX]) {
         if (!register_split_fits(kern)) return NVFP4_ERR_CUDA;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
           return NVFP4_ERR_CUDA;
-        info->gemm_attr_set[EPI + 4 * MX] = true;
+        info->gemm_attr_set[EPI + kEpiKinds * MX] = true;
       }
     }
     const int grid = args.num_tiles < info->sm_count ? args.num_tiles : info->sm_count;
@@ -215,17 +216,17 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   int max_clusters;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!info->pair_attr_set[EPI + 4 * MX]) {
+    if (!info->pair_attr_set[EPI + kEpiKinds * MX]) {
       if (!register_split_fits(kern)) return NVFP4_ERR_CUDA;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM_BYTES) != cudaSuccess)
         return NVFP4_ERR_CUDA;
       cfg.gridDim = dim3(2 * (info->sm_count / 2), 1, 1);
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return NVFP4_ERR_CUDA;
-      info->pair_clusters[EPI + 4 * MX] = n;
-      info->pair_attr_set[EPI + 4 * MX] = true;
+      info->pair_clusters[EPI + kEpiKinds * MX] = n;
+      info->pair_attr_set[EPI + kEpiKinds * MX] = true;
     }
-    max_clusters = info->pair_clusters[EPI + 4 * MX];
+    max_clusters = info->pair_clusters[EPI + kEpiKinds * MX];
   }
   const int clusters = args.num_tiles < max_clusters ? args.num_tiles : max_clusters;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
@@ -380,6 +381,21 @@ NVFP4_API nvfp4_status gemm_nvfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, cons
     args.q_cols = static_cast<int>(B.rows);
   }
   return run_gemm<nvfp4::EPI_POINTWISE>(A, B, D, ldd, B.rows, args, stream);
+}
+
+NVFP4_API nvfp4_status gemm_nvfp4_reduce_rows_f32(nvfp4_tensor A, nvfp4_tensor B, float* const* dst, int world,
+                                                  int64_t rows_per_rank, int64_t ldd, cudaStream_t stream) {
+  if (dst == nullptr || (reinterpret_cast<uintptr_t>(dst) & 7u) != 0) return NVFP4_ERR_INVALID_ARG;
+  if (world < 1 || rows_per_rank <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (rows_per_rank % 128 != 0 || A.rows != static_cast<int64_t>(world) * rows_per_rank)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (ldd < B.rows) return NVFP4_ERR_INVALID_ARG;
+  if (ldd % 4 != 0) return NVFP4_ERR_MISALIGNED;
+  nvfp4::GemmArgs args{};
+  args.red_dst = dst;
+  args.red_rows = rows_per_rank;
+  args.red_ldd = ldd;
+  return run_gemm<nvfp4::EPI_REDUCE>(A, B, nullptr, 0, B.rows, args, stream);
 }
 
 NVFP4_API int64_t mxfp4_sf_bytes(int64_t rows, int64_t cols) {

@@ -299,6 +299,14 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(x), "r"(y)
       : "memory");
 }
+// *addr += v, four floats, as one relaxed atomic at system scope: the address may be another
+// GPU's memory mapped into this one (peer access); .sys makes the addition well defined there.
+__device__ __forceinline__ void red_add_v4_f32(float* addr, const uint4& v) {
+  asm volatile("red.relaxed.sys.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(v.x)),
+               "f"(__uint_as_float(v.y)), "f"(__uint_as_float(v.z)), "f"(__uint_as_float(v.w))
+               : "memory");
+}
+
 // Per-warpgroup register budgets (all four warps of a warpgroup execute these together):
 // the role warps give registers back, the epilogue warpgroups take them.
 template <uint32_t N>

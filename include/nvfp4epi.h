@@ -201,6 +201,29 @@ nvfp4_status gemm_nvfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* b
                                   cudaStream_t stream);
 
 /*
+ * Row-parallel GEMM with its reduce-scatter in the epilogue. "Serving sub-second Ideogram v4
+ * without quality loss", section "Epilogue fusion in brief", applies the op following a GEMM
+ * to the accumulator so that no second pass runs. Here the op is the sum across ranks that
+ * follows a GEMM over one rank's slice of K: the down projection of a tensor-parallel FFN
+ * block.
+ *   C = G_A * G_B * (A B^T)     (float32, M x N, this rank's partial sum)
+ *   row m of C is added atomically into  dst[m / rows_per_rank] + (m % rows_per_rank) * ldd,
+ *   so destination r receives rows [r * rows_per_rank, (r + 1) * rows_per_rank).
+ *   dst: a DEVICE array of `world` float pointers, 8-byte aligned. Each pointer addresses a
+ *        rows_per_rank x N float32 block with leading dimension ldd (in floats, a multiple
+ *        of 4; pointers 16-byte aligned). A pointer may be another GPU's memory mapped into
+ *        this one (peer access); the additions are relaxed atomics at system scope.
+ *   The caller zeroes (or seeds) the destinations before the first rank's call, and reads
+ *   them only after every rank's call has completed: the call itself synchronises nothing.
+ *   Summation order across ranks is unspecified.
+ * Rules: the plain rules for A and B; A.rows == world * rows_per_rank, rows_per_rank a
+ *        multiple of 128 (UNSUPPORTED_SHAPE otherwise); ldd >= N (INVALID_ARG), ldd % 4 == 0
+ *        (MISALIGNED).
+ */
+nvfp4_status gemm_nvfp4_reduce_rows_f32(nvfp4_tensor A, nvfp4_tensor B, float* const* dst, int world,
+                                        int64_t rows_per_rank, int64_t ldd, cudaStream_t stream);
+
+/*
  * As gemm_nvfp4_plain, then per row and per head of head_dim adjacent columns among the
  * first n_norm_cols: y = x * rsqrt(mean(x^2) + eps) * w[col] (x = G_A G_B acc, float32);
  * columns >= n_norm_cols pass through (the V block of a QKV projection).

@@ -82,6 +82,14 @@ def test_argument_checks_return_status_without_gpu(lib):
     assert lib.rmsnorm_heads_bf16(16, 4, 256, 16, 256, 100, 1e-6, 16, 256, None) == SHAPE
     assert lib.swiglu_bf16(16, 4, 12, 24, 16, 12, None) == SHAPE
     assert lib.nvfp4_selftest_bounded_wait(0, None) == INVALID
+    # row-parallel reduce: destinations array, ranks, rows per rank, pitch
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), None, 2, 128, 256, None) == INVALID
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 12, 2, 128, 256, None) == INVALID  # dst % 8
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 0, 128, 256, None) == INVALID
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 4, 64, 256, None) == SHAPE  # rows % 128
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 1, 128, 256, None) == SHAPE  # M != w*rows
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 2, 128, 200, None) == INVALID  # ldd < N
+    assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 2, 128, 258, None) == MISALIGNED
 
 
 def test_valid_call_without_a_gpu_fails_loudly(lib):
