@@ -13,13 +13,18 @@ touching the epilogues:
   [r Nh/w, (r+1) Nh/w) of both the gate and the up half; its shard is interleaved as a
   whole, so SwiGLU stays inside each thread. No collective.
 - FFN-down, row-parallel: rank r multiplies its intermediate columns by the matching K
-  slice of the down weight, writing float32 partial sums (pointwise epilogue, f32 cast);
-  one NCCL reduce-scatter over the token rows sums them, leaving rank r the output rows
-  [r M/w, (r+1) M/w).
+  slice of the down weight; the partial sums over the ranks are added up, leaving rank r
+  the output rows [r M/w, (r+1) M/w). Two ways:
+  - reduce="nccl": the GEMM writes float32 partials (pointwise epilogue, f32 cast), then
+    one NCCL reduce-scatter over the token rows;
+  - reduce="fused": the GEMM's epilogue adds each partial row straight into its owner's
+    output block (gemm_nvfp4_reduce_rows_f32). The blocks are symmetric memory, so every
+    rank holds the others' addresses. A barrier before the GEMM means every block is
+    zeroed; a barrier after it means every addition has landed. The only traffic between
+    GPUs is those stores: no kernel loads from another GPU's memory.
 
 The index helpers below are pure host logic (tested with gloo ranks on the CPU); TPLayer
-runs them with the library's kernels and NCCL. No load in any kernel reads another GPU's
-memory: the only exchange is the NCCL reduce-scatter.
+runs them with the library's kernels and NCCL or symmetric memory.
 """
 from __future__ import annotations
 
@@ -77,7 +82,7 @@ class TPLayer:
     returns (qkv_local bf16 M x 3*(heads/w)*head_dim, out_rows float32 (M/w) x K)."""
 
     def __init__(self, w_qkv, w_up, w_down, w_norm_q, w_norm_k, heads: int, head_dim: int,
-                 h_gscale: float, group=None, eps: float = 1e-6):
+                 h_gscale: float, group=None, eps: float = 1e-6, reduce: str = "nccl"):
         import torch
         import torch.distributed as dist
         from . import _lib as L
@@ -103,6 +108,10 @@ class TPLayer:
         self.w_norm = torch.cat([w_norm_q.repeat(hr), w_norm_k.repeat(hr)]).float().contiguous().to(dev)
         self.h_gscale = float(h_gscale)
         self.nh_local = nh // self.world
+        if reduce not in ("nccl", "fused"):
+            raise ValueError(f"reduce must be 'nccl' or 'fused', not {reduce!r}")
+        self.reduce = reduce
+        self._fused = {}  # M -> (this rank's output block, symmetric-memory handle or None, pointers)
 
     def _pack(self, whole, shard, interleave: bool = False):
         T, L = self.L.NVFP4Tensor, self.L
@@ -122,6 +131,13 @@ class TPLayer:
         h = L.NVFP4Tensor.empty(M, self.nh_local, dev)
         h.gscale.fill_(self.h_gscale)  # static scale, the same on every rank
         L.gemm_nvfp4_swiglu(xq, self.Wup, None, h)
+        if self.reduce == "fused":
+            out, hdl, ptrs = self._fused_block(M, dev)
+            out.zero_()
+            self._barrier(hdl)  # every rank's block is zeroed before any rank adds into it
+            L.gemm_nvfp4_reduce_rows_f32(h, self.Wdown, ptrs, M // self.world, self.Wdown.rows)
+            self._barrier(hdl)  # every rank's additions have landed
+            return qkv, out
         part = torch.empty(M, self.Wdown.rows, dtype=torch.float32, device=dev)
         L.gemm_nvfp4_pointwise(h, self.Wdown, part)
         out = torch.empty(M // self.world, self.Wdown.rows, dtype=torch.float32, device=dev)
@@ -130,3 +146,29 @@ class TPLayer:
         else:
             out = part
         return qkv, out
+
+    def _fused_block(self, M: int, dev):
+        """This rank's (M/w) x N float32 output block and every rank's block address, made
+        once per M. With more than one rank the blocks are symmetric memory: each rank maps
+        the others' blocks and receives their addresses at the rendezvous."""
+        if M not in self._fused:
+            torch = self.torch
+            rows = output_rows(M, self.world, self.rank)
+            n = self.Wdown.rows
+            if self.world > 1:
+                import torch.distributed._symmetric_memory as symm_mem
+                block = symm_mem.empty((rows.stop - rows.start, n), dtype=torch.float32, device=dev)
+                hdl = symm_mem.rendezvous(block, self.group if self.group is not None else self.dist.group.WORLD)
+                ptrs = torch.tensor(list(hdl.buffer_ptrs), dtype=torch.int64, device=dev)
+            else:
+                block = torch.empty(rows.stop - rows.start, n, dtype=torch.float32, device=dev)
+                hdl = None
+                ptrs = torch.tensor([block.data_ptr()], dtype=torch.int64, device=dev)
+            self._fused[M] = (block, hdl, ptrs)
+        return self._fused[M]
+
+    def _barrier(self, hdl):
+        """Stream-ordered barrier over the ranks' symmetric memory (nothing to wait for at
+        world size 1)."""
+        if hdl is not None:
+            hdl.barrier(channel=0)

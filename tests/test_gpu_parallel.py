@@ -1,6 +1,7 @@
 """TPLayer on one GPU (no process group: world size 1) computes exactly what the
 unsharded kernels do: the shard packing with the whole weights' scales, the QKV shard's
-normalised-column count and the f32 partial-sum path of the row-parallel down GEMM."""
+normalised-column count and both row-parallel down paths (f32 partials for an NCCL
+reduce-scatter, and the reduction fused into the GEMM's epilogue)."""
 import numpy as np
 import pytest
 import torch
@@ -13,8 +14,8 @@ from gpu_util import device
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("M", [256, 384])
-def test_tp_layer_world1_equals_the_unsharded_kernels(M):
+@pytest.mark.parametrize("M,reduce", [(256, "nccl"), (384, "nccl"), (256, "fused"), (384, "fused")])
+def test_tp_layer_world1_equals_the_unsharded_kernels(M, reduce):
     dev = device()
     heads, hd, K, nh = 4, 128, 512, 512
     x = wk.activations(M, K, 1, seed=M).to(dev)
@@ -26,8 +27,9 @@ def test_tp_layer_world1_equals_the_unsharded_kernels(M):
     T = ep.NVFP4Tensor
     xq = ep.nvfp4_quantize(x, T.empty(M, K, dev))
     G_h = 0.01
-    layer = TPLayer(wq, wu, wd, wn_q, wn_k, heads, hd, G_h)
+    layer = TPLayer(wq, wu, wd, wn_q, wn_k, heads, hd, G_h, reduce=reduce)
     qkv, out = layer.step(xq)
+    qkv, out = layer.step(xq)  # a second step reuses (and re-zeroes) the fused output block
 
     Wq = ep.nvfp4_quantize(wq, T.empty(wq.shape[0], K, dev))
     Wu = ep.nvfp4_quantize(wu, T.empty(wu.shape[0], K, dev), interleave=True)
