@@ -390,6 +390,7 @@ def run_cuda(args):
         d32 = torch.empty(M, K_IN, dtype=torch.float32, device=dev)
         dq = ep.NVFP4Tensor.empty(M, K_IN, dev)
         dq.gscale.fill_(float(layer.out.float().abs().max().item()) / 2688)
+        red_ptrs = torch.tensor([d32.data_ptr()], dtype=torch.int64, device=dev)
         barrier()
         cases = {
             "plain_bf16": lambda: ep.gemm_nvfp4_plain(layer.h, layer.Wdown, layer.out),
@@ -397,6 +398,9 @@ def run_cuda(args):
             "bias_f32": lambda: ep.gemm_nvfp4_pointwise(layer.h, layer.Wdown, d32, bias=bias),
             "bias_relu_nvfp4_only": lambda: ep.gemm_nvfp4_pointwise(layer.h, layer.Wdown, None, bias=bias, relu=True,
                                                                    Dq=dq),
+            # the row-parallel down GEMM with its reduction fused in, into this GPU's own block
+            # (world size 1): atomic float32 additions instead of the f32 TMA stores above
+            "reduce_rows_f32": lambda: ep.gemm_nvfp4_reduce_rows_f32(layer.h, layer.Wdown, red_ptrs, M, K_IN),
         }
         pw = {}
         for name, fn in cases.items():
