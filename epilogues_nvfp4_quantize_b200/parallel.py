@@ -169,6 +169,7 @@ class TPLayer:
 
     def _barrier(self, hdl):
         """Stream-ordered barrier over the ranks' symmetric memory (nothing to wait for at
-        world size 1)."""
+        world size 1). Bounded: a rank that never arrives ends the wait after 10 s instead of
+        holding the others forever."""
         if hdl is not None:
-            hdl.barrier(channel=0)
+            hdl.barrier(channel=0, timeout_ms=10_000)
