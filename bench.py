@@ -333,7 +333,7 @@ def run_cuda(args):
                    "parallelism": f"dp{world} (independent token batches, no collective)",
                    "l2": "no flush: per-step inputs (x 100.7 MB + packed weights 75 MB) exceed the 126 MB L2"},
         "roofline": {"bound": "tensor",
-                     "kernel": ("gemm_nvfp4_pair_kernel<EPI_SWIGLU>" if M % 256 == 0 else
+                     "kernel": ("gemm_nvfp4_pair_kernel<EPI_SWIGLU>" if M > 128 else
                                 "gemm_nvfp4_kernel<EPI_SWIGLU>") + " (FFN-up, SwiGLU + NVFP4 re-quantisation)",
                      "achieved": round(up_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(up_tflops / fp4_peak, 4),

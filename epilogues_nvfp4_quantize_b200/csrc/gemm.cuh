@@ -5,11 +5,13 @@
 // output; the small op is applied to the accumulator and the result is written once.
 //
 // Two kernels share the epilogue:
-//   gemm_nvfp4_pair_kernel  (M % 256 == 0) a cluster of 2 CTAs on the two SMs of a TPC
-//       runs one 256 x 256 output tile with the pair MMA (tcgen05 cta_group::2): each CTA
-//       stages its own 128 rows of A and 128 of the 256 rows of B, so a CTA moves
-//       38 KB per K step of 256 for 128 x 256 x 256 MMA work (5-stage ring);
-//   gemm_nvfp4_kernel       (M % 256 == 128) one CTA per 128 x 256 tile (3-stage ring).
+//   gemm_nvfp4_pair_kernel  (M > 128) a cluster of 2 CTAs on the two SMs of a TPC runs
+//       one 256 x 256 output tile with the pair MMA (tcgen05 cta_group::2): each CTA stages
+//       its own 128 rows of A and 128 of the 256 rows of B, so a CTA moves 38 KB per K
+//       step of 256 for 128 x 256 x 256 MMA work (5-stage ring). When M % 256 == 128 the
+//       last tile's second CTA lies past M: its loads start past the end of A and of its
+//       scales and read zeros, its TMA stores are clipped, and its plain stores are skipped.
+//   gemm_nvfp4_kernel       (M == 128) one CTA per 128 x 256 tile (3-stage ring).
 // Warp roles (512 threads): warps 0-7 epilogue, warp 8 TMA producer, warp 9 TMEM owner
 // and MMA issuer, warps 10-13 copy the block scales from shared memory into TMEM
 // (tcgen05.cp), warps 14-15 idle. The role warpgroups run on 64 registers a thread and the
@@ -299,11 +301,13 @@ __device__ __forceinline__ void stage_row_bf16(uint8_t* box, int lane, const uin
   }
 }
 
-// Make the staging box visible to the TMA engine and store it at (x, y).
-__device__ __forceinline__ void flush_box(const CUtensorMap* map, uint8_t* box, int lane, int x, int y) {
+// Make the staging box visible to the TMA engine and store it at (x, y). A box whose first
+// row is at or past `rows` (the second half of a pair tile that ends past M) is not stored.
+__device__ __forceinline__ void flush_box(const CUtensorMap* map, uint8_t* box, int lane, int x, int y,
+                                          int rows) {
   fence_proxy_async_smem();
   __syncwarp();
-  if (lane == 0) {
+  if (lane == 0 && y < rows) {
     tma_store_2d(map, box, x, y);
     bulk_commit();
   }
@@ -393,9 +397,9 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
     if (args.write_d) {
       box_reuse_wait(lane);
       stage_row_bf16(c.box, lane, packed);
-      flush_box(c.tmD, c.box, lane, oc0, m0 + c.sub * 32);
+      flush_box(c.tmD, c.box, lane, oc0, m0 + c.sub * 32, args.M);
     }
-    if (args.q_codes != nullptr) {
+    if (args.q_codes != nullptr && m0 < args.M) {
       const int64_t row = m0 + row_in_tile;
       uint4* dst = reinterpret_cast<uint4*>(args.q_codes + row * (args.q_cols >> 1) + (oc0 >> 1));
       dst[0] = make_uint4(qc[0], qc[1], qc[2], qc[3]);
@@ -406,6 +410,7 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
   } else if constexpr (EPI == EPI_REDUCE) {
     // Row-parallel GEMM with its reduce-scatter fused in: this warp's 32 rows all belong to
     // one destination (red_rows is a multiple of 128), into which alpha * acc is added.
+    if (m0 >= args.M) return true;  // the second half of a last pair tile that ends past M
     const int64_t row0 = m0 + c.sub * 32;
     const int64_t owner = row0 / args.red_rows;
     float* dst = args.red_dst[owner] + (row0 - owner * args.red_rows) * args.red_ldd + col0;
@@ -440,7 +445,7 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
         for (int q = 0; q < 4; ++q) {
           box_reuse_wait(lane);
           stage_row_bf16(c.box, lane, v[q]);  // 32 words: 32 floats of the row
-          flush_box(c.tmD, c.box, lane, col0 + 32 * q, m0 + c.sub * 32);
+          flush_box(c.tmD, c.box, lane, col0 + 32 * q, m0 + c.sub * 32, args.M);
         }
       } else {
 #pragma unroll
@@ -454,11 +459,11 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
           }
           box_reuse_wait(lane);
           stage_row_bf16(c.box, lane, p);
-          flush_box(c.tmD, c.box, lane, col0 + 64 * h, m0 + c.sub * 32);
+          flush_box(c.tmD, c.box, lane, col0 + 64 * h, m0 + c.sub * 32, args.M);
         }
       }
     }
-    if (args.q_codes != nullptr) {
+    if (args.q_codes != nullptr && m0 < args.M) {
       const int64_t row = m0 + row_in_tile;
       uint4* dst = reinterpret_cast<uint4*>(args.q_codes + row * (args.q_cols >> 1) + (col0 >> 1));
 #pragma unroll
@@ -540,7 +545,7 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
       }
       box_reuse_wait(lane);
       stage_row_bf16(c.box, lane, p);
-      flush_box(c.tmD, c.box, lane, col0 + 64 * h, m0 + c.sub * 32);
+      flush_box(c.tmD, c.box, lane, col0 + 64 * h, m0 + c.sub * 32, args.M);
     }
     return true;
   }

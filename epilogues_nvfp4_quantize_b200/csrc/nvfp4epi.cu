@@ -116,8 +116,9 @@ nvfp4_status check_operand(const nvfp4_tensor& t) {
   return NVFP4_OK;
 }
 
-// Common checks and launch of the GEMM kernels: the CTA-pair kernel when M % 256 == 0,
-// the single-CTA kernel otherwise.
+// Common checks and launch of the GEMM kernels: the CTA-pair kernel from M = 256 on (for
+// M % 256 == 128 its last tile's second CTA computes rows past M, which are zeros and are
+// not stored), the single-CTA kernel for M = 128.
 template <int EPI, bool MX = false>
 nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int64_t ldd, int64_t n_out,
                       nvfp4::GemmArgs args, cudaStream_t stream) {
@@ -139,7 +140,7 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   DeviceInfo* info;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
 
-  const bool pair = (M % 256) == 0;
+  const bool pair = M > BM;
   CUtensorMap tmA, tmB, tmD, tmSFA, tmSFB;
   std::memset(&tmD, 0, sizeof(tmD));
   if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, A.codes, K / 2, M, K / 2, BK_BYTES, BM,
@@ -173,7 +174,7 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
   args.M = static_cast<int>(M);
   args.N = static_cast<int>(N);
   args.K = static_cast<int>(K);
-  args.tiles_m = static_cast<int>(M / (pair ? 256 : BM));
+  args.tiles_m = static_cast<int>(pair ? (M + 255) / 256 : M / BM);
   args.tiles_n = static_cast<int>(N / BN);
   args.num_tiles = args.tiles_m * args.tiles_n;
   // keep the smaller operand resident in L2 while the larger one streams through once

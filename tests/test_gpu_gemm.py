@@ -1,8 +1,9 @@
 """GPU parity of the fused GEMM entry points against the oracle, at sizes the oracle
 finishes in seconds that still span several tiles, several tiles per CTA, and the
-degenerate cases (one tile, one K step, no normalised columns). M % 256 == 0 runs the
-CTA-pair kernel, M % 256 == 128 the single-CTA kernel; both appear below, each with more
-tiles than the GPU has SMs (pairs) in at least one case."""
+degenerate cases (one tile, one K step, no normalised columns). From M = 256 on the CTA-pair
+kernel runs; for M % 256 == 128 its last tile's second CTA lies past M (rows 384, 1152, ...
+below). M = 128 runs the single-CTA kernel. Each appears with more tiles than the GPU has SMs
+(pairs) in at least one case."""
 import numpy as np
 import pytest
 import torch
@@ -42,21 +43,22 @@ def test_plain_gemm_is_exact_on_exactly_representable_inputs(M, N, K):
     assert np.array_equal(got, want), f"{int((got != want).sum())} of {got.size} outputs differ"
 
 
-@pytest.mark.parametrize("M", [8192, 8064])
-def test_plain_gemm_exact_over_many_ring_wraps(M):
-    """Many K steps per CTA (or CTA pair), about 35, through the 5-stage ring with 4 TMEM
-    scale slots (CTA pair, M = 8192) and the 3-stage ring with 3 slots (single CTA, M = 8064).
-    The stage and slot counters wrap against each other and across tile boundaries (4 K steps
-    per tile). Exactly representable inputs make every output bit-exact; rows are sampled,
+@pytest.mark.parametrize("M,N,K", [(8192, 5120, 1024), (8064, 5120, 1024), (128, 512, 4096)])
+def test_plain_gemm_exact_over_many_ring_wraps(M, N, K):
+    """Many K steps per CTA (or CTA pair) through the rings: about 35 in the 5-stage ring with
+    4 TMEM scale slots of the CTA pair (M = 8192, 4 K steps per tile; M = 8064 adds a last
+    tile half past M), and 16 in the 3-stage ring with 3 slots of the single CTA (M = 128,
+    one tile per CTA). The stage and slot counters wrap against each other and across tile
+    boundaries. Exactly representable inputs make every output bit-exact; rows are sampled,
     always including the first and the last."""
-    N, K = 5120, 1024
     qa, sa, qb, sb = _exact_operands(M, N, K, seed=77)
     A = nvfp4_from_arrays(qa, sa, 1.0)
     B = nvfp4_from_arrays(qb, sb, 1.0)
     D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
     ep.gemm_nvfp4_plain(A, B, D)
     rng = np.random.default_rng(M)
-    rows = np.sort(np.concatenate([[0, M - 1], rng.choice(np.arange(1, M - 1), size=254, replace=False)]))
+    n = min(256, M)
+    rows = np.sort(np.concatenate([[0, M - 1], rng.choice(np.arange(1, M - 1), size=n - 2, replace=False)]))
     ref = o.bf16_round(o.gemm(o.dequantize(qa[rows], sa[rows], 1.0), o.dequantize(qb, sb, 1.0)))
     got = bf16_bits(D[torch.from_numpy(rows).to(device())])
     want = o.bf16_bits(ref)
@@ -107,6 +109,8 @@ def _rmsnorm_case(M, K, N, hd, n_norm, seed=0, eps=1e-6):
     (256, 512, 768, 128, 384),      # 128-wide heads, normalised part ends mid-tile
     (384, 256, 512, 128, 0),        # nothing normalised
     (2048, 512, 2560, 256, 1536),   # several tiles per CTA
+    (128, 512, 768, 256, 512),      # the single-CTA kernel
+    (1152, 512, 1024, 256, 768),    # the pair kernel's last tile half past M
 ])
 def test_rmsnorm_gemm_matches_oracle(M, K, N, hd, n_norm):
     got, ref = _rmsnorm_case(M, K, N, hd, n_norm)

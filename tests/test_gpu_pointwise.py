@@ -1,8 +1,8 @@
 """GPU parity of gemm_nvfp4_pointwise (bias, ReLU, cast to bf16/f16/f32, optional NVFP4
 output for the next layer) against the oracle. Exactly representable operands make the
 FP32 accumulator exact, so the outputs are compared bit for bit; general operands within
-the benchmark spec's tolerance. M % 256 == 0 runs the CTA-pair kernel, M % 256 == 128 the
-single-CTA one."""
+the benchmark spec's tolerance. From M = 256 on the CTA-pair kernel runs (for M % 256 == 128 with
+its last tile half past M); M = 128 runs the single-CTA kernel."""
 import numpy as np
 import pytest
 import torch

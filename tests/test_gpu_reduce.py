@@ -27,11 +27,13 @@ def _operands(M, N, K, seed, exact):
     return quantize_gpu(a), quantize_gpu(b)
 
 
-# (world, rows per rank, N, K, exact operands): pair kernel (M % 256 == 0) and single-CTA
-# kernel (M % 256 == 128); 128 rows per rank puts the two halves of a pair tile on two ranks
+# (world, rows per rank, N, K, exact operands): M % 256 == 0, M % 256 == 128 (the last pair
+# tile half past M) and M = 128 (the single-CTA kernel); 128 rows per rank puts the two
+# halves of a pair tile on two ranks
 @pytest.mark.parametrize("world,rpr,N,K,exact", [(1, 256, 512, 512, True), (2, 256, 512, 1024, True),
                                                  (4, 128, 768, 512, True), (1, 384, 256, 256, True),
-                                                 (3, 384, 512, 512, True), (2, 1024, 1536, 1024, False)])
+                                                 (3, 384, 512, 512, True), (2, 1024, 1536, 1024, False),
+                                                 (1, 128, 512, 512, True)])
 def test_reduce_rows_equals_pointwise_f32(world, rpr, N, K, exact):
     M = world * rpr
     A, B = _operands(M, N, K, seed=world * 100 + rpr, exact=exact)
