@@ -413,7 +413,14 @@ __device__ __forceinline__ bool epilogue_tile(EpiCtx& c, int m0, int n0, Release
     if (m0 >= args.M) return true;  // the second half of a last pair tile that ends past M
     const int64_t row0 = m0 + c.sub * 32;
     const int64_t owner = row0 / args.red_rows;
-    float* dst = args.red_dst[owner] + (row0 - owner * args.red_rows) * args.red_ldd + col0;
+    float* const block = args.red_dst[owner];
+    // the host cannot see the pointer array: a destination that is not 16-byte aligned is
+    // reported in the device status word (NVFP4_ERR_MISALIGNED) and skipped, not dereferenced
+    if ((reinterpret_cast<uintptr_t>(block) & 15u) != 0) {
+      if (lane == 0) record_status(3, 60);
+      return true;
+    }
+    float* dst = block + (row0 - owner * args.red_rows) * args.red_ldd + col0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
 #pragma unroll

@@ -212,7 +212,10 @@ nvfp4_status gemm_nvfp4_pointwise(nvfp4_tensor A, nvfp4_tensor B, const float* b
  *   dst: a DEVICE array of `world` float pointers, 8-byte aligned. Each pointer addresses a
  *        rows_per_rank x N float32 block with leading dimension ldd (in floats, a multiple
  *        of 4; pointers 16-byte aligned). A pointer may be another GPU's memory mapped into
- *        this one (peer access); the additions are relaxed atomics at system scope.
+ *        this one (peer access); the additions are relaxed atomics at system scope. The host
+ *        cannot read the array: a pointer that is not 16-byte aligned is found by the kernel,
+ *        which skips that block's rows and records NVFP4_ERR_MISALIGNED for
+ *        nvfp4_read_device_status.
  *   The caller zeroes (or seeds) the destinations before the first rank's call, and reads
  *   them only after every rank's call has completed: the call itself synchronises nothing.
  *   Summation order across ranks is unspecified.

@@ -79,3 +79,22 @@ def test_reduce_rows_sums_k_slices_into_the_full_product():
 def _read(t):
     from gpu_util import read_nvfp4
     return read_nvfp4(t)
+
+
+def test_reduce_rows_misaligned_destination_is_reported_not_dereferenced():
+    """A destination pointer that is not 16-byte aligned cannot be checked on the host (the
+    pointer array is device memory): the kernel reports it in the device status word and
+    leaves that block alone; the aligned destination is still written."""
+    M, N, K = 256, 256, 256
+    A, B = _operands(M, N, K, seed=9, exact=True)
+    ref = torch.empty(M, N, dtype=torch.float32, device=device())
+    ep.gemm_nvfp4_pointwise(A, B, ref)
+    good = torch.zeros(128, N, dtype=torch.float32, device=device())
+    backing = torch.zeros(128 * N + 4, dtype=torch.float32, device=device())
+    bad_ptr = backing.data_ptr() + 4  # 4-byte offset: misaligned for the 16-byte additions
+    ptrs = torch.tensor([good.data_ptr(), bad_ptr], dtype=torch.int64, device=device())
+    ep.gemm_nvfp4_reduce_rows_f32(A, B, ptrs, 128, N)
+    assert ep.read_device_status() == 3  # NVFP4_ERR_MISALIGNED
+    assert torch.equal(good, ref[:128])
+    assert torch.all(backing == 0)
+    assert ep.read_device_status() == 0  # reading clears it
