@@ -27,7 +27,9 @@
  *     CUDA launch errors return NVFP4_ERR_CUDA. There is no exception, no abort and no
  *     device assert. Every wait inside a kernel is bounded in time; a wait that runs
  *     out records NVFP4_ERR_DEVICE_TIMEOUT in a device status word, read with
- *     nvfp4_read_device_status().
+ *     nvfp4_read_device_status(). The same word holds the one argument error that only
+ *     a kernel can see: a misaligned destination in gemm_nvfp4_reduce_rows_f32's device
+ *     pointer array (NVFP4_ERR_MISALIGNED).
  *   - Only compute capability 10.0 (B200) is supported (NVFP4_ERR_UNSUPPORTED_DEVICE).
  *   - bf16 tensors are row-major with a leading dimension given in elements.
  */
