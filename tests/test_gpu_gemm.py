@@ -145,7 +145,7 @@ def _swiglu_case(M, K, nh, seed=0, requant=True, write_d=True):
     return a, b, ref, G, D, Dq
 
 
-@pytest.mark.parametrize("M,K,nh", [(128, 256, 128), (256, 512, 512), (2048, 512, 1280)])
+@pytest.mark.parametrize("M,K,nh", [(128, 256, 128), (256, 512, 512), (2048, 512, 1280), (640, 512, 384)])
 def test_swiglu_gemm_matches_oracle(M, K, nh):
     a, b, ref, G, D, Dq = _swiglu_case(M, K, nh)
     got = bf16_to_np(D)
@@ -166,11 +166,13 @@ def test_swiglu_gemm_matches_oracle(M, K, nh):
     assert np.all(lv[code_diff] <= 2.0)
 
 
-def test_fused_requant_equals_quantize_of_fused_bf16():
+@pytest.mark.parametrize("M", [512, 384])
+def test_fused_requant_equals_quantize_of_fused_bf16(M):
     """GPU invariant: the re-quantised output is nvfp4_quantize (static scale) applied to
-    the fused bf16 output, bit for bit."""
-    a, b, ref, G, D, Dq = _swiglu_case(512, 768, 768, seed=4)
-    t = ep.NVFP4Tensor.empty(512, 768, device())
+    the fused bf16 output, bit for bit (M = 384: the last pair tile half past M, whose
+    re-quantised rows must not be written)."""
+    a, b, ref, G, D, Dq = _swiglu_case(M, 768, 768, seed=4)
+    t = ep.NVFP4Tensor.empty(M, 768, device())
     t.gscale.fill_(float(G))
     ep.nvfp4_quantize(D, t, compute_amax=False)
     q1, s1, _, b1 = read_nvfp4(Dq)
@@ -229,3 +231,28 @@ def test_bounded_wait_times_out_into_a_status_and_the_context_survives():
 def test_no_device_errors_recorded():
     torch.cuda.synchronize()
     assert ep.read_device_status() == 0
+
+
+def test_rmsnorm_and_swiglu_respect_a_padded_output_pitch():
+    """Outputs written into a wider buffer (leading dimension > N): the values match the
+    contiguous results bit for bit and the columns past N stay untouched. M = 384 also puts
+    the last pair tile half past M."""
+    M, K, N, hd, nn = 384, 512, 768, 256, 512
+    a = wk.activations(M, K, wk.outlier_count(K), seed=12)
+    b = wk.weights(N, K, 1 / np.sqrt(K), seed=12)
+    w = np.tile(wk.norm_weight(hd, 12), nn // hd).astype(np.float32)
+    A, B = quantize_gpu(a), quantize_gpu(b)
+    wt = torch.from_numpy(w).to(device())
+    D = torch.empty(M, N, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_rmsnorm(A, B, wt, hd, nn, 1e-6, D)
+    Dp = torch.full((M, N + 64), 3.0, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_rmsnorm(A, B, wt, hd, nn, 1e-6, Dp[:, :N])
+    assert torch.equal(Dp[:, :N], D)
+    assert torch.all(Dp[:, N:] == 3.0)
+    Bi = quantize_gpu(b, interleave=True)
+    Y = torch.empty(M, N // 2, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_swiglu(A, Bi, Y, None)
+    Yp = torch.full((M, N // 2 + 128), 3.0, dtype=torch.bfloat16, device=device())
+    ep.gemm_nvfp4_swiglu(A, Bi, Yp[:, :N // 2], None)
+    assert torch.equal(Yp[:, :N // 2], Y)
+    assert torch.all(Yp[:, N // 2:] == 3.0)
