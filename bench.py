@@ -600,28 +600,48 @@ def _blas_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(M: int, rows: int = 256):
+def _timed_rows(layer, sample, chunk=1024):
+    """Seconds for the oracle step over `sample`, run in row chunks so memory stays bounded."""
+    t0 = time.perf_counter()
+    for i in range(0, len(sample), chunk):
+        layer.step(sample[i:i + chunk])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(M: int, rows: int = 0, target_s: float = 10.0):
+    """The oracle timed on a bounded sample of the step's rows. rows=0 sizes the sample by time:
+    a 256-row probe, then enough rows for about `target_s` seconds of CPU work (at most M). One
+    core is timed the same way with a third of the target."""
     layer = OracleLayer(M)
     rng = np.random.default_rng(0)
-    sample = np.sort(rng.choice(M, size=rows, replace=False))
-    t0 = time.perf_counter()
-    layer.step(sample)
-    dt = time.perf_counter() - t0
-    fl = sum(step_flops(rows).values())
+    order = rng.permutation(M)
+
+    def pick(n):
+        return np.sort(order[:n])
+
+    def sized(budget):
+        probe = min(256, M)
+        d = _timed_rows(layer, pick(probe))
+        if rows:
+            n = min(rows, M)
+        else:
+            n = min(M, max(probe, int(probe * budget / max(d, 1e-6)) // 64 * 64))
+        if n == probe:
+            return n, d
+        return n, _timed_rows(layer, pick(n))
+
+    n, dt = sized(target_s)
+    fl = sum(step_flops(n).values())
     out = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-           "sample": f"{rows} random rows of the M={M} step (quantise, fp64 GEMMs, RMSNorm, SwiGLU, requant, "
+           "sample": f"{n} random rows of the M={M} step (quantise, fp64 GEMMs, RMSNorm, SwiGLU, requant, "
                      f"down GEMM) in {dt:.2f} s; weight packing ({layer.pack_s:.1f} s, once per model) excluded",
            "host_threads": os.cpu_count()}
-    # the same oracle on one core, on a quarter of the sample
     try:
         from threadpoolctl import threadpool_limits
-        r1 = max(8, rows // 4)
         with threadpool_limits(limits=1):
-            t0 = time.perf_counter()
-            layer.step(sample[:r1])
-            d1 = time.perf_counter() - t0
-        out["one_core"] = {"value": round(sum(step_flops(r1).values()) / d1 / 1e12, 6), "unit": "TFLOP/s",
-                           "sample": f"{r1} rows in {d1:.2f} s"}
+            n1, d1 = sized(target_s / 3) if not rows else (max(8, n // 4), _timed_rows(layer, pick(max(8, n // 4))))
+        out["one_core"] = {"value": round(sum(step_flops(n1).values()) / d1 / 1e12, 6), "unit": "TFLOP/s",
+                           "sample": f"{n1} rows in {d1:.2f} s"}
     except ImportError:  # pragma: no cover
         pass
     return out
@@ -899,7 +919,8 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--M", type=int, default=16384, help="tokens per GPU per step")
     ap.add_argument("--cmp-steps", type=int, default=10, help="steps of each fused/unfused comparison loop")
-    ap.add_argument("--cpu-rows", type=int, default=256, help="rows of the oracle sample in cpu_baseline")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="rows of the oracle sample in cpu_baseline (0: as many as about 10 s of CPU work takes)")
     ap.add_argument("--ref-rows", type=int, default=64, help="rows per step of the --impl reference arm")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the FFN-up kernel from an ncu capture of this kernel")
