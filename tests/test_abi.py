@@ -92,6 +92,23 @@ def test_argument_checks_return_status_without_gpu(lib):
     assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 2, 128, 258, None) == MISALIGNED
 
 
+def test_empty_inputs_are_rejected_before_any_launch(lib):
+    """Zero rows or columns are a shape error on every entry point that takes sizes: the
+    kernels never see an empty grid."""
+    SHAPE = 2
+    assert lib.nvfp4_quantize(16, 0, 256, 256, 0, 0, _t(0, 256), None, None) == SHAPE
+    assert lib.nvfp4_quantize(16, 128, 0, 256, 0, 0, _t(128, 0), None, None) == SHAPE
+    assert lib.nvfp4_quantize_noalloc(16, 0, 256, 256, 0, _t(0, 256), None) == SHAPE
+    assert lib.nvfp4_fake_quantize(16, 0, 256, 256, 0, 16, 16, 256, None, None) == SHAPE
+    assert lib.mxfp4_quantize(16, 0, 256, 256, 0, _t(0, 256), None) == SHAPE
+    assert lib.gemm_nvfp4_plain(_t(0, 256), _t(256, 256), 16, 256, None) == SHAPE      # M = 0
+    assert lib.gemm_nvfp4_plain(_t(128, 256), _t(0, 256), 16, 256, None) == SHAPE      # N = 0
+    assert lib.gemm_nvfp4_plain(_t(128, 0), _t(256, 0), 16, 256, None) == SHAPE        # K = 0
+    assert lib.gemm_mxfp4_plain(_t(0, 256), _t(256, 256), 16, 256, None) == SHAPE
+    assert lib.rmsnorm_heads_bf16(16, 0, 256, 16, 128, 256, 1e-6, 16, 256, None) == SHAPE
+    assert lib.swiglu_bf16(16, 0, 16, 32, 16, 16, None) == SHAPE
+
+
 def test_valid_call_without_a_gpu_fails_loudly(lib):
     import torch
     if torch.cuda.is_available():
