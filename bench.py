@@ -608,11 +608,12 @@ def _timed_rows(layer, sample, chunk=1024):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(M: int, rows: int = 0, target_s: float = 10.0):
+def cpu_baseline(M: int, rows: int = 0, target_s: float = 10.0, layer=None):
     """The oracle timed on a bounded sample of the step's rows. rows=0 sizes the sample by time:
     a 256-row probe, then enough rows for about `target_s` seconds of CPU work (at most M). One
-    core is timed the same way with a third of the target."""
-    layer = OracleLayer(M)
+    core is timed the same way with a third of the target. `layer`: an OracleLayer of M rows
+    (built here when None)."""
+    layer = OracleLayer(M) if layer is None else layer
     rng = np.random.default_rng(0)
     order = rng.permutation(M)
 
