@@ -141,3 +141,45 @@ def test_pointwise_matches_torch_float32_bias_add_and_relu():
     # ReLU zeroes exactly the negative sums
     y = o.pointwise(c, bias)
     assert np.array_equal(o.pointwise(c, bias, relu=True) == 0, y <= 0)
+
+
+def _ab(M, N, K, seed):
+    return wk.activations(M, K, 1, seed), wk.weights(N, K, 1 / np.sqrt(K), seed)
+
+
+def test_problem_swiglu_is_odd_in_the_up_half_only():
+    """silu(g) * u is odd in u and not in g. Quantisation is sign-symmetric (sign-magnitude
+    codes, scales from |x|), so negating the up rows of B negates the output exactly, while
+    negating the gate rows does not: a composition that swapped the halves fails."""
+    M, Nh, K = 6, 32, 64
+    a, b = _ab(M, 2 * Nh, K, 7)
+    base = o.problem_swiglu(a, b)
+    neg_up = torch.cat([b[:Nh], -b[Nh:]])
+    np.testing.assert_array_equal(o.problem_swiglu(a, neg_up), -base)
+    neg_gate = torch.cat([-b[:Nh], b[Nh:]])
+    assert not np.array_equal(o.problem_swiglu(a, neg_gate), -base)
+    assert base.shape == (M, Nh)
+
+
+def test_problem_rmsnorm_is_invariant_to_a_power_of_two_scale_of_a():
+    """Doubling A doubles G and leaves every code and block scale unchanged, so C doubles
+    exactly. With eps = 0 the normalised heads do not move, and the passthrough (V) columns
+    double exactly (bf16 rounding commutes with a power of two)."""
+    M, N, K, hd = 4, 512, 256, 128
+    a, b = _ab(M, N, K, 9)
+    w = np.random.default_rng(1).uniform(0.5, 1.5, 256)
+    y1 = o.problem_rmsnorm(a, b, w, hd, 256, 0.0)
+    y2 = o.problem_rmsnorm(a * 2, b, w, hd, 256, 0.0)
+    np.testing.assert_array_equal(y2[:, :256], y1[:, :256])
+    np.testing.assert_array_equal(y2[:, 256:], 2 * y1[:, 256:])
+    np.testing.assert_array_equal(y1[:, 256:], o.problem_plain(a, b)[:, 256:])
+
+
+def test_problem_pointwise_relu_is_the_positive_part_of_the_same_sum():
+    M, N, K = 5, 64, 128
+    a, b = _ab(M, N, K, 11)
+    bias = np.random.default_rng(2).standard_normal(N).astype(np.float32)
+    y = o.problem_pointwise(a, b, bias)
+    r = o.problem_pointwise(a, b, bias, relu=True)
+    np.testing.assert_array_equal(r, np.maximum(y, 0.0))
+    assert (y < 0).any() and (r >= 0).all()
