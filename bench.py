@@ -43,6 +43,23 @@ def step_flops(M: int) -> dict:
     return {"qkv": 2 * M * N_QKV * K_IN, "up": 2 * M * N_UP * K_IN, "down": 2 * M * K_DOWN * K_IN}
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over the ranks of the default process group (x itself with one rank).
+    The whole job's time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Work of all ranks per step over the slowest rank's time per step, in TFLOP/s."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def workload_desc(M: int) -> str:
     return (f"DiT layer projections at M={M} tokens: quantise x ({M}x{K_IN} bf16) -> QKV GEMM "
             f"N={N_QKV} + per-head RMSNorm hd{HD} on Q,K (V passthrough) -> FFN-up GEMM N={N_UP} "
@@ -293,11 +310,7 @@ def run_cuda(args):
         stop.record()
         torch.cuda.synchronize(dev)
     launches = ep.launch_count() - n0
-    ms_total = start.elapsed_time(stop)
-    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(stop), dev)
     ms_step = ms_total / K
     per = {"quantize_x": [], "qkv_rmsnorm": [], "up_swiglu_requant": [], "down_plain": []}
     for i in range(K):
@@ -306,7 +319,7 @@ def run_cuda(args):
         per["up_swiglu_requant"].append(ev[i][1].elapsed_time(ev[i][2]))
         per["down_plain"].append(ev[i][2].elapsed_time(ev_e[i]))
     avg = {k: sum(v) / len(v) for k, v in per.items()}
-    value = total_flops * world / (ms_total / K * 1e-3) / 1e12
+    value = whole_job_tflops(total_flops, world, ms_step)
     clocks = clk.summary()
 
     pk = peaks()
@@ -529,13 +542,9 @@ def run_cuda(args):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e2e_steps(n_e2e, e0, e1)
         torch.cuda.synchronize(dev)
-        t_e2e = e0.elapsed_time(e1) / n_e2e
-        te = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        t_e2e = float(te.item())
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
         ok = torch.equal(out_host[(n_e2e - 1) & 1], layer.out.cpu()) if world == 1 else None
-        result["e2e"] = {"value": round(total_flops * world / (t_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        result["e2e"] = {"value": round(whole_job_tflops(total_flops, world, t_e2e), 2), "unit": "TFLOP/s",
                          "h2d_bytes_per_step": int(x_host.numel() * 2),
                          "d2h_bytes_per_step": int((qkv_host[0].numel() + out_host[0].numel()) * 2),
                          "ms_per_step": round(t_e2e, 4), "steps": n_e2e,
