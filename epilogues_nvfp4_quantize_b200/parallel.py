@@ -79,7 +79,9 @@ class TPLayer:
 
     Weights are given whole (bf16, on this rank's device) and sharded here; each rank
     packs only its shard. step(xq) takes the NVFP4 activations (replicated, M x K) and
-    returns (qkv_local bf16 M x 3*(heads/w)*head_dim, out_rows float32 (M/w) x K)."""
+    returns (qkv_local bf16 M x 3*(heads/w)*head_dim, out_rows float32 (M/w) x K).
+    With reduce="fused", out_rows is this rank's symmetric-memory block for that M: the next
+    step of the same M zeroes and refills it, so copy it out to keep it."""
 
     def __init__(self, w_qkv, w_up, w_down, w_norm_q, w_norm_k, heads: int, head_dim: int,
                  h_gscale: float, group=None, eps: float = 1e-6, reduce: str = "nccl"):
