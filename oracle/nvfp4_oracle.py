@@ -20,10 +20,22 @@ It is the plain definition of what the path computes, written from
 
 The NVFP4 block format (16 elements along K share one unsigned E4M3 scale, one FP32
 scale per tensor) is not spelled out on the page; the oracle uses that reading, with
-the per-tensor scale G = amax / (6 * 448) so that the largest block scale lands on the
-largest E4M3 value. Every quantisation decision (which code, which scale) is taken in
-IEEE float32, in the exact operation order stated in ``quantize``; the GEMM,
-normalisation and activation are evaluated in float64 on the decoded values and
+the per-tensor scale G = amax / (6 * 448) (an FP32 number) so that the largest block
+scale lands on the largest E4M3 value.
+
+Two statements of the quantiser live here:
+
+* ``quantize`` is the plain definition: the block scale is the E4M3 value nearest to
+  amax_b / (6 G) and each code the E2M1 value nearest to x / d, both decided on the exact
+  quotients (ties to the even code). It is the oracle's answer.
+* ``quantize_fp32_order`` takes the same decisions through IEEE float32 reciprocals and
+  products, the order a GPU evaluates cheaply. Its results differ from the plain
+  definition only where a quotient lies within ``TIE_REL`` of a rounding midpoint;
+  ``quantize_ties`` marks those places. Tests compare a GPU result with the plain
+  definition (codes and scales may differ only at those ties) and, bit for bit, with the
+  float32 order.
+
+The GEMM, normalisation and activation are evaluated in float64 on the decoded values and
 rounded once to bfloat16 (round to nearest even).
 
 Everything here is pinned by ``tests/test_oracle_*.py`` against closed forms, library
@@ -80,18 +92,19 @@ def _rne_to_table(ax: np.ndarray, table: np.ndarray) -> np.ndarray:
 
 
 def e2m1_encode(x) -> np.ndarray:
-    """float32 -> E2M1 code, round to nearest with ties to the even mantissa,
-    saturating at +-6. The sign bit follows the input's sign bit (so -0.1 -> 0x8).
+    """Real number (float32 or float64) -> E2M1 code, round to nearest with ties to the
+    even mantissa, saturating at +-6. The sign bit follows the input's sign bit (so
+    -0.1 -> 0x8).
 
     The magnitude index is the number of midpoints between adjacent levels that |x|
     lies above; at a midpoint exactly, the even index of the two neighbours wins.
-    (Every midpoint is exact in float32, so the comparisons are exact.)
+    (Every midpoint is exact in binary floating point, so the comparisons are exact.)
     """
-    x = np.asarray(x, dtype=F32)
+    x = np.asarray(x, dtype=np.float64)
     ax = np.abs(x)
     idx = np.zeros(x.shape, np.uint8)
     for i in range(7):
-        mid = F32((_E2M1_MAGS[i] + _E2M1_MAGS[i + 1]) / 2)
+        mid = (_E2M1_MAGS[i] + _E2M1_MAGS[i + 1]) / 2
         idx += (ax > mid)
         if (i + 1) % 2 == 0:
             idx += (ax == mid)
@@ -121,8 +134,9 @@ _E4M3_TABLE = e4m3_decode(np.arange(256))        # code -> value lookup
 
 
 def e4m3_encode(x) -> np.ndarray:
-    """Non-negative float32 -> E4M3 code, round to nearest even, saturating at 448."""
-    ax = np.asarray(x, dtype=F32).astype(np.float64)
+    """Non-negative real number (float32 or float64) -> E4M3 code, round to nearest
+    even, saturating at 448 (infinity saturates too)."""
+    ax = np.asarray(x, dtype=np.float64)
     if np.any(ax < 0) or np.any(np.isnan(ax)):
         raise ValueError("block scales are non-negative numbers")
     return _rne_to_table(ax, _E4M3_MAGS).astype(np.uint8)
@@ -142,27 +156,87 @@ def global_scale(x) -> np.float32:
     return F32(amax / GLOBAL_DIV)
 
 
-def quantize(x, G=None):
-    """Quantise a (rows, cols) float32 tensor to NVFP4, blocks of 16 along cols.
-
-    Steps, each an IEEE float32 operation in this order:
-      G    = amax(|x|) / 2688                (unless a static G is given)
-      enc  = 1 / (6 * G)
-      per block of 16:  amax_b = max |x_i|
-      s    = E4M3_rne_sat(amax_b * enc)     (s = 0 when amax_b == 0)
-      d    = dec(s) * G
-      r    = 1 / d
-      q_i  = E2M1_rne_sat(x_i * r)          (q_i = 0 when d == 0)
-    The decoded value of element i is dec(q_i) * dec(s) * G.
-
-    Returns (codes uint8 (rows, cols), scales uint8 (rows, cols/16), G float32).
-    """
+def _blocks(x):
     x = np.asarray(x, dtype=F32)
     rows, cols = x.shape
     if cols % BLOCK:
         raise ValueError("cols must be a multiple of 16")
+    return x, x.reshape(rows, cols // BLOCK, BLOCK)
+
+
+def quantize(x, G=None):
+    """Quantise a (rows, cols) float32 tensor to NVFP4, blocks of 16 along cols: the plain
+    definition.
+
+      G    = fp32(amax(|x|) / 2688)           (unless a static G is given)
+      per block of 16:  amax_b = max |x_i|
+      s    = E4M3_rne_sat(amax_b / (6 G))     (0 when amax_b == 0)
+      d    = dec(s) * G
+      q_i  = E2M1_rne_sat(x_i / d)            (0 when d == 0)
+
+    The decoded value of element i is dec(q_i) * dec(s) * G.
+
+    Both roundings are decided on the exact quotient. The quotients are formed in float64,
+    which decides them exactly: d has at most 28 significant bits (4 of dec(s), 24 of G)
+    and 6 G at most 26, so a float32 numerator is either exactly on a rounding midpoint
+    (at most 5 significant bits) times the denominator, or at least 2^-31 (relative) away
+    from it, far more than float64's 2^-53 rounding of the quotient. dec(s) * G is exact
+    in float64.
+
+    Returns (codes uint8 (rows, cols), scales uint8 (rows, cols/16), G float32).
+    """
+    x, blocks = _blocks(x)
+    rows, cols = x.shape
     G = global_scale(x) if G is None else F32(G)
-    blocks = x.reshape(rows, cols // BLOCK, BLOCK)
+    amax_b = np.max(np.abs(blocks), axis=2).astype(np.float64) if cols else np.zeros((rows, 0))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(amax_b > 0, amax_b / (6.0 * float(G)), 0.0)   # +inf when G == 0
+    s = e4m3_encode(ratio)
+    return codes_for_scales(x, s, G), s, G
+
+
+def _quotients(x, s, G):
+    """x_i / d per element (float64) and d > 0 per block, d = dec(s) * G (exact)."""
+    x, blocks = _blocks(x)
+    d = e4m3_decode(s) * float(G)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = blocks.astype(np.float64) / np.where(d > 0, d, 1.0)[:, :, None]
+    return v, d > 0
+
+
+def codes_for_scales(x, s, G) -> np.ndarray:
+    """The element step of ``quantize`` for given block scale codes s:
+    q_i = E2M1_rne_sat(x_i / (dec(s) * G)), 0 where that scale is 0."""
+    v, pos = _quotients(x, s, G)
+    q = np.where(pos[:, :, None], e2m1_encode(v), np.uint8(0)).astype(np.uint8)
+    return q.reshape(np.shape(x))
+
+
+def code_ties_for_scales(x, s, G) -> np.ndarray:
+    """Elements whose quotient x_i / (dec(s) * G) lies within TIE_REL of an E2M1
+    midpoint, for given block scale codes s."""
+    v, pos = _quotients(x, s, G)
+    return (_near_midpoint(v, _E2M1_MIDS) & pos[:, :, None]).reshape(np.shape(x))
+
+
+def quantize_fp32_order(x, G=None):
+    """The same quantiser with every step an IEEE float32 operation, in this order:
+
+      G    = fp32(amax(|x|) / 2688)            (unless a static G is given)
+      enc  = 1 / (6 * G)
+      s    = E4M3_rne_sat(amax_b * enc)       (0 when amax_b == 0)
+      d    = dec(s) * G
+      r    = 1 / d
+      q_i  = E2M1_rne_sat(x_i * r)            (0 when d == 0)
+
+    Each of 6 G, enc and amax_b * enc (and of d, r and x_i * r) rounds once, so the float32
+    quotient is within 3 * 2^-24 (relative) of the exact one, and a decision can differ from
+    ``quantize`` only where the exact quotient lies that close to a rounding midpoint
+    (``quantize_ties`` marks every such place). Same return values as ``quantize``.
+    """
+    x, blocks = _blocks(x)
+    rows, cols = x.shape
+    G = global_scale(x) if G is None else F32(G)
     amax_b = np.max(np.abs(blocks), axis=2) if cols else np.zeros((rows, 0), F32)
     with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
         enc = F32(F32(1.0) / F32(F32(6.0) * G)) if G != 0 else F32(np.inf)
@@ -175,6 +249,50 @@ def quantize(x, G=None):
     q = e2m1_encode(v)
     q = np.where((d > 0)[:, :, None], q, np.uint8(0)).astype(np.uint8)
     return q.reshape(rows, cols), s, G
+
+
+# A quotient within this relative distance of a rounding midpoint is a tie: 8 * 2^-24,
+# more than the 3 * 2^-24 that three float32 roundings (a reciprocal-multiply order) can
+# move it, so any float32 evaluation order of the quotient agrees with the exact
+# decision everywhere else.
+TIE_REL = 2.0 ** -21
+
+_E2M1_MIDS = (_E2M1_MAGS[:-1] + _E2M1_MAGS[1:]) / 2
+_E4M3_MIDS = (_E4M3_MAGS[:-1] + _E4M3_MAGS[1:]) / 2
+
+
+def _near_midpoint(v, mids, rel=TIE_REL) -> np.ndarray:
+    """|v| within rel (relative) of one of the midpoints."""
+    av = np.abs(np.asarray(v, np.float64))
+    if len(mids) > 16:   # long tables: only the two nearest midpoints can be that close
+        hi = np.clip(np.searchsorted(mids, av), 1, len(mids) - 1)
+        lo = hi - 1
+        return (np.abs(av - mids[lo]) <= rel * mids[lo]) | (np.abs(av - mids[hi]) <= rel * mids[hi])
+    out = np.zeros(av.shape, bool)
+    for m in mids:
+        out |= np.abs(av - m) <= rel * m
+    return out
+
+
+def quantize_ties(x, G=None):
+    """Where the quantisation of x is a tie (section-5 reading of the quantiser: both
+    neighbouring results are correct there). Returns (block_tie (rows, cols/16),
+    elem_tie (rows, cols)):
+
+      block_tie: amax_b / (6 G) lies within TIE_REL of a midpoint between two E4M3 values,
+                 so the block's scale may round either way;
+      elem_tie:  x_i / d (d from the plain definition's scale) lies within TIE_REL of a
+                 midpoint between two E2M1 levels.
+    """
+    x, blocks = _blocks(x)
+    rows, cols = x.shape
+    G = global_scale(x) if G is None else F32(G)
+    q, s, _ = quantize(x, G)
+    amax_b = np.max(np.abs(blocks), axis=2).astype(np.float64) if cols else np.zeros((rows, 0))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(amax_b > 0, amax_b / (6.0 * float(G)), 0.0)
+    block_tie = _near_midpoint(np.where(np.isfinite(ratio), ratio, 0.0), _E4M3_MIDS)
+    return block_tie, code_ties_for_scales(x, s, G)
 
 
 def dequantize(codes, scales, G) -> np.ndarray:
@@ -190,15 +308,43 @@ def fake_quantize(x, G=None):
     """Quantise-dequantise ("fake quantisation" of quantisation-aware distillation, page
     "Serving sub-second Ideogram v4 without quality loss", section on quantization-aware
     distillation): the forward pass sees the FP4 rounding noise. Returns (y, G) with
-    y = bf16(fp32(e2m1(q) * e4m3(s)) * fp32 G): the level-scale product is exact in fp32,
-    the product with G is one fp32 rounding, the result is rounded to bf16 (RNE).
+    y = bf16(dec(q) * dec(s) * G), the dequantised value of the plain quantiser rounded
+    once to bf16 (RNE; the product has at most 30 significant bits, exact in float64).
     The backward pass (straight-through estimator) is the identity and needs no oracle."""
     q, s, G = quantize(x, G)
+    return bf16_round(dequantize(q, s, G)), G
+
+
+def fake_quantize_fp32_order(x, G=None):
+    """The float32 evaluation order of fake quantisation: codes from
+    ``quantize_fp32_order``, y = bf16(fp32(fp32(e2m1(q) * e4m3(s)) * G)). The level-scale
+    product is exact in float32; its product with G rounds once to float32 and then to
+    bf16, which can differ from ``fake_quantize`` only at the ties ``fake_quantize_ties``
+    marks."""
+    q, s, G = quantize_fp32_order(x, G)
     rows, cols = q.shape
     ls = (_E2M1_TABLE[q & 0xF].reshape(rows, cols // BLOCK, BLOCK)
           * _E4M3_TABLE[np.asarray(s)][:, :, None]).reshape(rows, cols)
     y32 = ls.astype(np.float32) * np.float32(G)
     return bf16_round(y32.astype(np.float64)), G
+
+
+def _near_bf16_midpoint(v, rel=2.0 ** -23) -> np.ndarray:
+    """|v| within rel (relative) of a midpoint between two adjacent bf16 values (where a
+    float32 intermediate rounding can decide the bf16 rounding differently)."""
+    m, _ = np.frexp(np.abs(np.asarray(v, np.float64)))   # |v| = m * 2^e, 0.5 <= m < 1
+    t = m * 256.0                                         # bf16 ulps: 128 <= t < 256
+    return (np.abs(t - (np.floor(t) + 0.5)) <= rel * t) & (m > 0)
+
+
+def fake_quantize_ties(x, G=None) -> np.ndarray:
+    """Elements of fake_quantize(x, G) where both neighbouring bf16 results are correct:
+    a code tie, any element of a block whose scale is a tie, or a dequantised value within
+    2^-23 (relative) of a bf16 rounding midpoint."""
+    bt, et = quantize_ties(x, G)
+    q, s, G = quantize(x, G)
+    near = _near_bf16_midpoint(dequantize(q, s, G))
+    return et | np.repeat(bt, BLOCK, axis=1) | near
 
 
 # ----------------------------------------------------------------------------------
@@ -445,6 +591,17 @@ def mx_quantize(x):
     return q, e
 
 
+def mx_codes_for_scales(y, e8m0) -> np.ndarray:
+    """The element step of ``mx_quantize`` for given E8M0 scale codes:
+    E2M1_rn_satfinite(y / 2^(e - 127)), 0 in blocks whose code is 0."""
+    y = np.asarray(y, dtype=F32)
+    rows, cols = y.shape
+    X = e8m0_decode(e8m0)[:, :, None]
+    q = e2m1_encode(y.reshape(rows, cols // MX_BLOCK, MX_BLOCK).astype(np.float64) / X)
+    q = np.where((np.asarray(e8m0) > 0)[:, :, None], q, np.uint8(0)).astype(np.uint8)
+    return q.reshape(rows, cols)
+
+
 def mx_dequantize(codes, e8m0) -> np.ndarray:
     """dec(q) * 2^(e - 127) in float64, (rows, cols)."""
     codes = np.asarray(codes)
@@ -454,11 +611,36 @@ def mx_dequantize(codes, e8m0) -> np.ndarray:
     return vals.reshape(rows, cols)
 
 
+def _hadamard_matrix(n: int) -> np.ndarray:
+    """Unnormalised Sylvester-Hadamard matrix of order n (a power of two): the Kronecker
+    product H2 (x) H2 (x) ... of the 2 x 2 matrix [[1, 1], [1, -1]]."""
+    h2 = np.array([[1.0, 1.0], [1.0, -1.0]])
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.kron(h2, h)
+    return h
+
+
+H32 = _hadamard_matrix(MX_BLOCK)
+
+
 def hadamard32(x) -> np.ndarray:
-    """x @ H32 per block of 32 along cols, H32 the unnormalised Sylvester-Hadamard matrix
-    (entries +-1), computed in float32 by the fast Walsh-Hadamard transform: five stages,
+    """x @ H32 per block of 32 along cols: a float64 matrix product with the Kronecker
+    matrix H32 (entries +-1), rounded once to float32. H32 H32^T = 32 I, so
+    (x H)(w H)^T = 32 x w^T. (The float64 sums of 32 float32 terms are exact unless a
+    block's magnitudes span more than 2^24.)"""
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    y = x.reshape(rows, cols // MX_BLOCK, MX_BLOCK).astype(np.float64) @ H32
+    return y.reshape(rows, cols).astype(F32)
+
+
+def hadamard32_fp32_order(x) -> np.ndarray:
+    """The same transform as the fast Walsh-Hadamard butterfly in float32: five stages,
     stage h in (1, 2, 4, 8, 16) maps each pair (j, j + h), j with bit h clear, to
-    (a + b, a - b). H32 H32^T = 32 I, so (x H)(w H)^T = 32 x w^T."""
+    (a + b, a - b), each sum rounded to float32. After k stages an output's error is at
+    most k * 2^-24 * S, S the block's sum of |x_i|, so it lies within 6 * 2^-24 * S of
+    ``hadamard32``'s result."""
     x = np.asarray(x, dtype=F32)
     rows, cols = x.shape
     y = x.reshape(rows, cols // MX_BLOCK, MX_BLOCK).copy()
@@ -470,6 +652,36 @@ def hadamard32(x) -> np.ndarray:
         y[:, :, :, 1, :] = a - b
         h *= 2
     return y.reshape(rows, cols)
+
+
+def mx_transform_ties(x, e8m0=None):
+    """Where the MXFP4 quantisation of hadamard32(x) is decided within the float32 error
+    of evaluating the transform (6 * 2^-24 * S, S the block's sum of |x_i|; the band is
+    8 * 2^-24 * S). Returns (block_tie (rows, cols/32), elem_tie (rows, cols)):
+
+      block_tie: the block's amax lies within the band of a power of two (its shared
+                 exponent may come out either way);
+      elem_tie:  y_i / X lies within band / X of an E2M1 midpoint (X the block scale of
+                 mx_quantize(hadamard32(x)), or the scales e8m0 when given).
+    """
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    nb = cols // MX_BLOCK
+    S = np.abs(x.reshape(rows, nb, MX_BLOCK).astype(np.float64)).sum(axis=2)
+    band = 8.0 * 2.0 ** -24 * S
+    y = hadamard32(x).reshape(rows, nb, MX_BLOCK).astype(np.float64)
+    amax = np.abs(y).max(axis=2)
+    with np.errstate(divide="ignore"):
+        p = np.round(np.log2(np.where(amax > 0, amax, 1.0)))
+    block_tie = (np.abs(amax - np.ldexp(1.0, p.astype(np.int64))) <= band) & (amax > 0)
+    e = mx_quantize(y.reshape(rows, cols).astype(F32))[1] if e8m0 is None else np.asarray(e8m0)
+    X = e8m0_decode(e)
+    v = np.abs(y) / X[:, :, None]
+    bx = (band / X)[:, :, None]
+    elem_tie = np.zeros(v.shape, bool)
+    for m in _E2M1_MIDS:
+        elem_tie |= np.abs(v - m) <= bx
+    return block_tie, elem_tie.reshape(rows, cols)
 
 
 def mx_sf_bytes(rows: int, cols: int) -> int:

@@ -11,8 +11,8 @@ import torch
 import epilogues_nvfp4_quantize_b200 as ep
 from oracle import nvfp4_oracle as o
 import workloads as wk
-from gpu_util import (assert_close, bf16_bits, bf16_to_np, device, nvfp4_from_arrays, quantize_gpu,
-                      read_nvfp4, rel_err, REL_TOL)
+from gpu_util import (assert_close, assert_requant_point13, bf16_bits, bf16_to_np, device, level_index,
+                      nvfp4_from_arrays, quantize_gpu, read_nvfp4, rel_err, REL_TOL)
 
 pytestmark = pytest.mark.gpu
 
@@ -150,20 +150,13 @@ def test_swiglu_gemm_matches_oracle(M, K, nh):
     a, b, ref, G, D, Dq = _swiglu_case(M, K, nh)
     got = bf16_to_np(D)
     assert_close(got, ref, "swiglu")
-    # re-quantised output, code for code against the oracle's re-quantisation of its
-    # own bf16 result: a differing code is allowed only where the two bf16 values differ,
-    # and then by at most one level
-    q_ref, s_ref, _ = o.requantize(ref, G)
+    # re-quantised output, code for code: the plain re-quantisation of the GPU's own bf16
+    # output up to ties; against the oracle's re-quantisation of its own bf16 result, a
+    # code or scale may differ only where the two bf16 values differ, by one level (one
+    # scale code)
     q, s, Gq, _ = read_nvfp4(Dq)
     assert Gq == G
-    same_bf16 = np.repeat((got == ref).reshape(M, nh // 16, 16).all(axis=2), 16, axis=1)
-    code_diff = q != q_ref
-    assert not (code_diff & same_bf16).any()
-    blk_same = (got == ref).reshape(M, nh // 16, 16).all(axis=2)
-    assert np.array_equal(s[blk_same], s_ref[blk_same])
-    lv = np.abs(o.e2m1_decode(q) - o.e2m1_decode(q_ref))
-    assert code_diff.mean() < 0.01
-    assert np.all(lv[code_diff] <= 2.0)
+    assert assert_requant_point13(q, s, got, ref, G, "swiglu requant") < 0.01
 
 
 @pytest.mark.parametrize("M", [512, 384])
@@ -184,6 +177,12 @@ def test_swiglu_requant_only():
     a, b, ref, G, D, Dq = _swiglu_case(256, 256, 256, seed=6, write_d=False)
     q_ref, s_ref, _ = o.requantize(ref, G)
     q, s, _, _ = read_nvfp4(Dq)
+    # without the bf16 output to compare, the codes follow the oracle's up to one level and
+    # one scale code, and differ on few elements
+    assert np.all(np.abs(s.astype(int) - s_ref.astype(int)) <= 1)
+    same = np.repeat(s == s_ref, 16, axis=1)
+    assert np.all(np.abs(level_index(q) - level_index(q_ref))[same] <= 1)
+    assert (q != q_ref).mean() < 0.01
     deq = o.dequantize(q, s, G)
     deq_ref = o.dequantize(q_ref, s_ref, G)
     assert np.linalg.norm(deq - deq_ref) / np.linalg.norm(deq_ref) < 1e-2

@@ -1,5 +1,8 @@
-"""GPU parity of the MXFP4 path: mxfp4_quantize (with and without the 32-point block
-Hadamard transform) bit for bit against the oracle; the MXFP4 GEMM exact on exactly
+"""GPU parity of the MXFP4 path: mxfp4_quantize without the transform bit for bit against
+the oracle; with the 32-point block Hadamard transform, equal to the plain definition
+(x H32 exactly, rounded once to float32, then MXFP4) except where the float32 error of
+evaluating the transform decides a rounding, and bit for bit equal to the oracle's float32
+butterfly order; the MXFP4 GEMM exact on exactly
 representable operands (pins the E8M0 scale layout and the block32 MMA descriptor), and
 within tolerance on workload operands; the transform lowers the error on outlier
 channels, which is its purpose."""
@@ -29,12 +32,32 @@ def test_mx_quantize_matches_oracle_bitwise(rows, cols, hadamard):
     x = wk.activations(rows, cols, 3, seed=rows + cols)
     t = ep.mxfp4_quantize(x.to(device()), ep.NVFP4Tensor.empty_mx(rows, cols, device()), hadamard=hadamard)
     xf = x.float().numpy()
-    q_ref, e_ref = o.mx_quantize(o.hadamard32(xf) if hadamard else xf)
     q, e, g, buf = _read_mx(t)
+    if hadamard:
+        _check_transform_plain(q, e, xf)
+    q_ref, e_ref = o.mx_quantize(o.hadamard32_fp32_order(xf) if hadamard else xf)
     assert np.array_equal(e, e_ref), f"{int((e != e_ref).sum())} scale mismatches"
     assert np.array_equal(q, q_ref), f"{int((q != q_ref).sum())} code mismatches"
     assert np.array_equal(buf, o.mx_pack_scales(e_ref, cols))  # padding bytes are 0
     assert g == (float(np.float32(1 / np.sqrt(32))) if hadamard else 1.0)
+
+
+def _check_transform_plain(q, e, xf):
+    """Codes and E8M0 scales of the transformed tensor against the plain definition
+    mx_quantize(hadamard32(x)): a scale may differ only in a block whose amax is within
+    the transform's float32 error band of a power of two; codes only at element ties, or,
+    in a block whose scale took the other side, they are the plain rounding under the GPU's
+    scale."""
+    q_ref, e_ref = o.mx_quantize(o.hadamard32(xf))
+    bt, et = o.mx_transform_ties(xf)
+    ed = e != e_ref
+    assert not (ed & ~bt).any(), f"{int((ed & ~bt).sum())} scales differ outside a tie"
+    same = np.repeat(~ed, 32, axis=1)
+    assert not ((q != q_ref) & same & ~et).any(), "codes differ outside a tie"
+    if ed.any():
+        q_alt = o.mx_codes_for_scales(o.hadamard32(xf), e)
+        _, et_alt = o.mx_transform_ties(xf, e)
+        assert not ((q != q_alt) & ~same & ~et_alt).any(), "codes under a tie scale differ outside a tie"
 
 
 def _mx_from_arrays(codes, e8m0, g=1.0):
@@ -102,8 +125,10 @@ def test_mx_gemm_with_transform_matches_oracle_and_beats_no_transform_on_outlier
 def test_mx_quantize_interleaved_weight_bitwise():
     w = wk.weights(2 * 200, 256, 1 / 16, seed=21)
     t = ep.mxfp4_quantize(w.to(device()), ep.NVFP4Tensor.empty_mx(400, 256, device()), hadamard=True, interleave=True)
-    q_ref, e_ref = o.mx_quantize(o.hadamard32(o.interleave_gate_up(w.float().numpy())))
+    wi = o.interleave_gate_up(w.float().numpy())
     q, e, _, _ = _read_mx(t)
+    _check_transform_plain(q, e, wi)
+    q_ref, e_ref = o.mx_quantize(o.hadamard32_fp32_order(wi))
     assert np.array_equal(e, e_ref) and np.array_equal(q, q_ref)
 
 

@@ -1,7 +1,9 @@
 """TPLayer on one GPU (no process group: world size 1) computes exactly what the
 unsharded kernels do: the shard packing with the whole weights' scales, the QKV shard's
 normalised-column count and both row-parallel down paths (f32 partials for an NCCL
-reduce-scatter, and the reduction fused into the GEMM's epilogue)."""
+reduce-scatter, and the reduction fused into the GEMM's epilogue). Its outputs are also
+checked against the oracle's layer: QKV with per-head RMSNorm, and the FFN chain (SwiGLU,
+static re-quantisation, down projection) in float64."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +11,8 @@ import torch
 import epilogues_nvfp4_quantize_b200 as ep
 from epilogues_nvfp4_quantize_b200.parallel import TPLayer
 import workloads as wk
-from gpu_util import device
+from oracle import nvfp4_oracle as o
+from gpu_util import assert_close, device
 
 pytestmark = pytest.mark.gpu
 
@@ -45,3 +48,14 @@ def test_tp_layer_world1_equals_the_unsharded_kernels(M, reduce):
     assert torch.equal(qkv, qkv_ref)
     assert torch.equal(out, out_ref)
     assert ep.read_device_status() == 0
+
+    # the oracle's layer on the same inputs
+    xc, wqc, wuc, wdc = x.cpu(), wq.cpu(), wu.cpu(), wd.cpu()
+    w_norm_np = w_norm.cpu().numpy()
+    qkv_o = o.problem_rmsnorm(xc, wqc, w_norm_np, hd, 2 * heads * hd, 1e-6)
+    assert_close(qkv.float().cpu().numpy().astype(np.float64), qkv_o, "TPLayer QKV vs oracle")
+    h_o = o.problem_swiglu(xc, wuc)
+    qh, sh, _ = o.requantize(h_o, np.float32(G_h))
+    qd, sd, gd = o.quantized_operand(wdc)
+    out_o = o.gemm(o.dequantize(qh, sh, np.float32(G_h)), o.dequantize(qd, sd, gd))
+    assert_close(out.cpu().numpy().astype(np.float64), out_o, "TPLayer FFN vs oracle")

@@ -10,7 +10,7 @@ import torch
 import epilogues_nvfp4_quantize_b200 as ep
 from oracle import nvfp4_oracle as o
 import workloads as wk
-from gpu_util import assert_close, device, nvfp4_from_arrays, quantize_gpu, read_nvfp4
+from gpu_util import assert_close, assert_nvfp4_plain, device, nvfp4_from_arrays, quantize_gpu, read_nvfp4
 
 pytestmark = pytest.mark.gpu
 
@@ -81,6 +81,8 @@ def test_pointwise_nvfp4_output_equals_quantize_of_bf16_output(M):
     q1, s1, _, b1 = read_nvfp4(Dq)
     q2, s2, _, b2 = read_nvfp4(t)
     assert np.array_equal(q1, q2) and np.array_equal(b1, b2)
+    # and against the oracle: the plain quantisation of the bf16 output, up to ties
+    assert_nvfp4_plain(q1, s1, D.float().cpu().numpy(), np.float32(G), "pointwise nvfp4 output")
     Dq2 = ep.NVFP4Tensor.empty(M, N, device())
     Dq2.gscale.fill_(G)
     ep.gemm_nvfp4_pointwise(A, B, None, bias=bias, Dq=Dq2)

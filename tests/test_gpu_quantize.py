@@ -1,6 +1,10 @@
-"""GPU parity of nvfp4_quantize against the oracle: codes, block scales and the
-per-tensor scale must agree bit for bit (both sides take every decision with the same
-IEEE float32 operations)."""
+"""GPU parity of nvfp4_quantize against the oracle.
+
+- Against the plain definition (exact quotients): the per-tensor scale bit for bit; block
+  scales and codes equal except at rounding ties, where they may take the neighbouring
+  value (one code, one level).
+- Against the oracle's float32 evaluation order (reciprocal times x, the order the kernel
+  uses): codes, scales and padding bytes bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -8,7 +12,7 @@ import torch
 import epilogues_nvfp4_quantize_b200 as ep
 from oracle import nvfp4_oracle as o
 import workloads as wk
-from gpu_util import device, quantize_gpu, read_nvfp4
+from gpu_util import assert_nvfp4_plain, device, quantize_gpu, read_nvfp4
 
 pytestmark = pytest.mark.gpu
 
@@ -17,13 +21,15 @@ def _check_bitwise(x_bf16, t, G_static=None, interleave=False):
     x = x_bf16.float().numpy()
     if interleave:
         x = o.interleave_gate_up(x)
-    q_ref, s_ref, G_ref = o.quantize(x, G_static)
     q, s, G, buf = read_nvfp4(t)
+    G_ref = o.global_scale(x) if G_static is None else np.float32(G_static)
     assert G == G_ref
-    assert np.array_equal(s, s_ref), f"{int((s != s_ref).sum())} scale mismatches"
-    assert np.array_equal(q, q_ref), f"{int((q != q_ref).sum())} code mismatches"
+    assert_nvfp4_plain(q, s, x, G_ref, "nvfp4_quantize")
+    q32, s32, _ = o.quantize_fp32_order(x, G_static)
+    assert np.array_equal(s, s32), f"{int((s != s32).sum())} scale mismatches (float32 order)"
+    assert np.array_equal(q, q32), f"{int((q != q32).sum())} code mismatches (float32 order)"
     # padding bytes of the scale buffer are zero
-    assert np.array_equal(buf, o.pack_scales(s_ref, x.shape[1]))
+    assert np.array_equal(buf, o.pack_scales(s32, x.shape[1]))
 
 
 @pytest.mark.parametrize("rows,cols,outliers", [(256, 1024, 8), (130, 192, 1), (1, 64, 0), (4096, 3072, 3)])
@@ -95,3 +101,20 @@ def test_quantize_reuses_workspace_across_calls():
         t = ep.NVFP4Tensor.empty(128, 256, device())
         ep.nvfp4_quantize(x.to(device()), t, workspace=ws)
         _check_bitwise(x, t)
+
+
+def test_quantize_ties_follow_the_float32_order_and_stay_within_the_tie_rule():
+    """Weights with their dynamic scale: G = amax / (6 * 448) turns many x / d into ratios
+    of short bf16 numbers that sit on a rounding midpoint except for the float32 rounding
+    of G (and amax_b / (6 G) = 448 * amax_b / amax, a ratio of two bf16 numbers, sits on a
+    scale midpoint the same way). For this seed the plain definition and the float32 order
+    disagree on about 1 % of the block scales and 0.3 % of the codes. The kernel must take
+    the float32 order's side there, inside the tie rule."""
+    w = wk.weights(2048, 3072, 1 / np.sqrt(3072), seed=3)
+    t = quantize_gpu(w)
+    q, s, G, _ = read_nvfp4(t)
+    wf = w.float().numpy()
+    exempt_scales, exempt_codes = assert_nvfp4_plain(q, s, wf, G, "weights")
+    assert exempt_scales > 0 and exempt_codes > 0
+    q32, s32, _ = o.quantize_fp32_order(wf)
+    assert np.array_equal(q, q32) and np.array_equal(s, s32)

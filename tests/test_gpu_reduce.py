@@ -2,7 +2,9 @@
 (gemm_nvfp4_reduce_rows_f32). Every destination lives on this GPU here: the kernel addresses a
 peer-mapped destination exactly as a local one, and the world sizes, row splits and pitches
 below cover its owner arithmetic. The reference is the pointwise GEMM's float32 output: the
-reduce epilogue computes the same G_A G_B acc, and adding it into zero is exact."""
+reduce epilogue computes the same G_A G_B acc, and adding it into zero is exact. Both are
+also checked against the oracle's float64 GEMM of the same codes: bit for bit on exactly
+representable operands, within the tolerance otherwise."""
 import numpy as np
 import pytest
 import torch
@@ -10,7 +12,7 @@ import torch
 import epilogues_nvfp4_quantize_b200 as ep
 from oracle import nvfp4_oracle as o
 import workloads as wk
-from gpu_util import device, nvfp4_from_arrays, quantize_gpu
+from gpu_util import assert_close, device, nvfp4_from_arrays, quantize_gpu, read_nvfp4
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +50,15 @@ def test_reduce_rows_equals_pointwise_f32(world, rpr, N, K, exact):
         assert torch.equal(outs[r][:, :N], ref[r * rpr:(r + 1) * rpr]), f"destination {r}"
         if ldd > N:
             assert torch.all(outs[r][:, N:] == 0), "columns past N are untouched"
+    # the oracle's float64 GEMM of the same codes and scales
+    qa, sa, ga, _ = read_nvfp4(A)
+    qb, sb, gb, _ = read_nvfp4(B)
+    full = o.gemm(o.dequantize(qa, sa, ga), o.dequantize(qb, sb, gb))
+    got = np.concatenate([t[:, :N].cpu().numpy() for t in outs]).astype(np.float64)
+    if exact:
+        assert np.array_equal(got, full.astype(np.float32).astype(np.float64))
+    else:
+        assert_close(got, full, "reduce rows vs oracle")
     # a second call adds the same values again: exactly twice the first result
     ep.gemm_nvfp4_reduce_rows_f32(A, B, ptrs, rpr, ldd)
     torch.cuda.synchronize()

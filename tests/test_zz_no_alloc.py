@@ -10,6 +10,7 @@ import torch
 
 import epilogues_nvfp4_quantize_b200 as ep
 from epilogues_nvfp4_quantize_b200 import _lib
+from oracle import nvfp4_oracle as o
 import workloads as wk
 
 
@@ -41,4 +42,14 @@ def test_noalloc_matches_workspace_quantiser_on_consecutive_calls(rows, cols, in
         assert torch.equal(got.gscale, ref.gscale)
         assert torch.equal(got.codes, ref.codes)
         assert torch.equal(got.sf, ref.sf)
+        # and against the oracle: the plain definition up to ties, the float32 order exactly
+        from gpu_util import assert_nvfp4_plain, read_nvfp4
+        xf = x.float().cpu().numpy()
+        if interleave:
+            xf = o.interleave_gate_up(xf)
+        q, s, G, _ = read_nvfp4(got)
+        assert G == o.global_scale(xf)
+        assert_nvfp4_plain(q, s, xf, G, "noalloc")
+        q32, s32, _ = o.quantize_fp32_order(xf)
+        assert np.array_equal(q, q32) and np.array_equal(s, s32)
     assert ep.read_device_status() == 0
