@@ -37,6 +37,7 @@ METRIC = "fused NVFP4 GEMM+epilogue TFLOPS and % of B200 FP4 peak; fused-vs-unfu
 K_IN, N_QKV, N_NORM, HD, N_UP, K_DOWN = 3072, 9216, 6144, 256, 24576, 12288
 EPS = 1e-6
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+FP4_DATASHEET_TFLOPS = 9000.0  # B200 dense FP4, the vendor's figure
 
 
 def step_flops(M: int) -> dict:
@@ -243,6 +244,38 @@ class Layer:
         ep.nvfp4_quantize(self.y_up, self.h2, compute_amax=False)
 
 
+def max_rel_err(got, ref) -> float:
+    """max |g - o| / max(|o|, 1e-2 rms(o)): the bf16 output tolerance rule of the tests."""
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    return float(np.max(np.abs(got - ref) / np.maximum(np.abs(ref), 1e-2 * rms))) if ref.size else 0.0
+
+
+def vendor_yardstick(layer, M, steps, torch, ep, flops):
+    """cuBLASLt NVFP4 (torch._scaled_mm) at the FFN-up and FFN-down shapes on the step's own
+    packed operands (the scale buffers already have the 128 x 4 tensor-core layout it
+    expects). Never a product path: it shows how much of the tensor pipe a vendor GEMM
+    without an epilogue gets on the same GPU."""
+    out = {"what": "torch._scaled_mm (cuBLASLt) NVFP4, bf16 out, no epilogue, same operands"}
+    try:
+        f4, f8 = torch.float4_e2m1fn_x2, torch.float8_e4m3fn
+        cases = {"ffn_up": (layer.xq, layer.Wup_logical, flops["up"]),
+                 "ffn_down": (layer.h, layer.Wdown, flops["down"])}
+        for name, (A, B, fl) in cases.items():
+            a = A.codes.view(f4)
+            b = B.codes.view(f4)
+            sa = A.sf.view(f8).view(A.rows, A.cols // 16)
+            sb = B.sf.view(f8).view(B.rows, B.cols // 16)
+            D = torch.empty(A.rows, B.rows, dtype=torch.bfloat16, device=A.codes.device)
+            t_v = time_loop(lambda: torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16), steps, 3, torch)
+            t_o = time_loop(lambda: ep.gemm_nvfp4_plain(A, B, D), steps, 3, torch)
+            out[name] = {"vendor_us": round(t_v * 1e3, 1), "vendor_tflops": round(fl / (t_v * 1e-3) / 1e12, 1),
+                         "ours_plain_us": round(t_o * 1e3, 1), "ours_tflops": round(fl / (t_o * 1e-3) / 1e12, 1)}
+            del D
+    except Exception as e:  # the vendor path is optional context, never required
+        out["error"] = f"{type(e).__name__}: {e}"[:200]
+    return out
+
+
 def time_loop(fn, steps, warmup, torch):
     for _ in range(warmup):
         fn()
@@ -289,10 +322,13 @@ def run_cuda(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # ---- warm-up
+    # ---- warm-up; its outputs are the reference of the timed steps' outputs (same inputs,
+    # deterministic kernels: every timed step must reproduce them bit for bit)
     for _ in range(args.warmup):
         layer.step()
     barrier()
+    qkv_warm, out_warm = layer.qkv.clone(), layer.out.clone()
+    ep.read_device_status()  # start the timed region with a clear status word
 
     # ---- timed region: K back-to-back steps (inputs x + weights exceed the L2)
     K = args.steps
@@ -310,6 +346,15 @@ def run_cuda(args):
         stop.record()
         torch.cuda.synchronize(dev)
     launches = ep.launch_count() - n0
+    # the timed steps checked themselves: no bounded wait gave up (device status word) and
+    # the last step's outputs equal the warm-up's
+    status = ep.read_device_status()
+    output_ok = bool(torch.equal(layer.qkv, qkv_warm) and torch.equal(layer.out, out_warm))
+    del qkv_warm, out_warm
+    check_rows = np.sort(np.random.default_rng([7, M]).choice(M, size=min(64, M), replace=False))
+    sel = torch.from_numpy(check_rows).to(dev)
+    last_qkv = layer.qkv[sel].float().cpu().numpy().astype(np.float64)
+    last_out = layer.out[sel].float().cpu().numpy().astype(np.float64)
     ms_total = max_over_ranks(start.elapsed_time(stop), dev)
     ms_step = ms_total / K
     per = {"quantize_x": [], "qkv_rmsnorm": [], "up_swiglu_requant": [], "down_plain": []}
@@ -358,7 +403,14 @@ def run_cuda(args):
         "kernels": kernels,
         "gpu_launches": launches,
         "clocks": clocks,
+        "status_ok": status == 0,
+        "output_ok": output_ok,
     }
+    result["roofline"]["peak_datasheet"] = FP4_DATASHEET_TFLOPS
+    result["roofline"]["frac_of_datasheet"] = round(up_tflops / FP4_DATASHEET_TFLOPS, 4)
+    for k in ("qkv_rmsnorm", "up_swiglu_requant", "down_plain"):
+        kernels[k]["pct_fp4_datasheet"] = round(100.0 * kernels[k]["tflops"] / FP4_DATASHEET_TFLOPS, 2)
+    kernels["quantize_x"]["pct_hbm"] = round(100.0 * kernels["quantize_x"]["gbs"] / pk["hbm_gbs"], 1)
 
     # ---- unfused comparison (separately timed, same step shapes)
     if not args.no_unfused:
@@ -444,6 +496,11 @@ def run_cuda(args):
         }
         del xm, wm, c_mx, c_nv, w_up_bf16
 
+    # ---- vendor yardstick: cuBLASLt's NVFP4 GEMM (torch._scaled_mm, no epilogue, bf16 out)
+    # on this step's own operands, against this library's plain GEMM of the same shapes
+    if not args.no_unfused:
+        result["yardstick"] = vendor_yardstick(layer, M, args.cmp_steps, torch, ep, flops)
+
     # ---- a small-batch step (serving): eager launches vs one CUDA-graph replay
     if not args.no_unfused:
         small = Layer(1024, dev, seed=rank + 100)
@@ -494,8 +551,16 @@ def run_cuda(args):
     # over three streams (host->device, compute, device->host) with two device buffer sets,
     # so the copies of neighbouring steps overlap this step's kernels (PCIe is full duplex).
     if not args.no_e2e:
+        import workloads as wk
         n_e2e = max(2, min(K // 2, 60))
-        x_host = layer.x.cpu().pin_memory()
+        # two different inputs alternate, so a step that read or returned a stale buffer
+        # would fail the output check; each input's outputs computed eagerly beforehand
+        x_host = [layer.x.cpu().pin_memory(),
+                  wk.activations(M, K_IN, wk.outlier_count(K_IN), seed=rank + 1000).pin_memory()]
+        ref_out = []
+        for xb in x_host:
+            layer.step(x=xb.to(dev))
+            ref_out.append((layer.qkv.cpu(), layer.out.cpu()))
         qkv_host = [torch.empty(layer.qkv.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         out_host = [torch.empty(layer.out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         x_dev = [layer.x, torch.empty_like(layer.x)]
@@ -517,7 +582,7 @@ def run_cuda(args):
                 with torch.cuda.stream(s_in):
                     if started[b]:
                         s_in.wait_event(ev_cmp[b])  # the compute of step i-2 has read x_dev[b]
-                    x_dev[b].copy_(x_host, non_blocking=True)
+                    x_dev[b].copy_(x_host[b], non_blocking=True)
                     ev_in[b].record(s_in)
                 with torch.cuda.stream(s_cmp):
                     s_cmp.wait_event(ev_in[b])
@@ -543,23 +608,39 @@ def run_cuda(args):
         e2e_steps(n_e2e, e0, e1)
         torch.cuda.synchronize(dev)
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dev)
-        ok = torch.equal(out_host[(n_e2e - 1) & 1], layer.out.cpu()) if world == 1 else None
+        ok = all(torch.equal(qkv_host[b], ref_out[b][0]) and torch.equal(out_host[b], ref_out[b][1])
+                 for b in (0, 1))
         result["e2e"] = {"value": round(whole_job_tflops(total_flops, world, t_e2e), 2), "unit": "TFLOP/s",
-                         "h2d_bytes_per_step": int(x_host.numel() * 2),
+                         "h2d_bytes_per_step": int(x_host[0].numel() * 2),
                          "d2h_bytes_per_step": int((qkv_host[0].numel() + out_host[0].numel()) * 2),
                          "ms_per_step": round(t_e2e, 4), "steps": n_e2e,
                          "pipelined": "3 streams (h2d, compute, d2h), 2 device buffer sets",
+                         "inputs": "two different host inputs, alternating",
                          "output_check": ok}
+        del ref_out
         del x_dev[1], qkv_dev[1], out_dev[1]
 
     if rank == 0 and world == 1 and not args.no_cpu:
-        result["cpu_baseline"] = cpu_baseline(M, rows=args.cpu_rows)
+        # the oracle checks the last timed step on seeded rows (the FFN activations
+        # re-quantised with the same static scale as the GPU's), then is timed as the CPU
+        # baseline
+        ol = OracleLayer(M)
+        ol.Gh = np.float32(layer.h.gscale.item())
+        qkv_o, out_o = ol.step(check_rows)
+        e_qkv, e_out = max_rel_err(last_qkv, qkv_o), max_rel_err(last_out, out_o)
+        result["oracle_check"] = {"rows": len(check_rows), "qkv_max_rel": round(e_qkv, 5),
+                                  "out_max_rel": round(e_out, 5), "tolerance": 2e-2,
+                                  "ok": bool(e_qkv <= 2e-2 and e_out <= 2e-2)}
+        result["cpu_baseline"] = cpu_baseline(M, rows=args.cpu_rows, layer=ol)
 
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result))
+    if not (result["status_ok"] and result["output_ok"]):
+        raise SystemExit(f"timed steps failed their self-check: status_ok={result['status_ok']} "
+                         f"output_ok={result['output_ok']}")
 
 
 # ----------------------------------------------------------------------------------

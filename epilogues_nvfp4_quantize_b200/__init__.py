@@ -28,5 +28,6 @@ from ._lib import (  # noqa: F401
     rmsnorm_heads_bf16,
     selftest_bounded_wait,
     sf_bytes,
+    signal_barrier,
     swiglu_bf16,
 )

@@ -26,7 +26,7 @@ EXPORTS = (
     "nvfp4_read_device_status", "nvfp4_selftest_bounded_wait", "nvfp4_launch_count",
     "nvfp4_quantize_noalloc", "nvfp4_fake_quantize", "gemm_nvfp4_pointwise",
     "mxfp4_sf_bytes", "mxfp4_quantize", "gemm_mxfp4_pointwise", "gemm_mxfp4_plain",
-    "gemm_mxfp4_rmsnorm", "gemm_mxfp4_swiglu", "gemm_nvfp4_reduce_rows_f32",
+    "gemm_mxfp4_rmsnorm", "gemm_mxfp4_swiglu", "gemm_nvfp4_reduce_rows_f32", "nvfp4_signal_barrier",
 )
 
 
@@ -70,6 +70,7 @@ def load() -> ctypes.CDLL:
         "gemm_mxfp4_plain": (i32, [_Tensor, _Tensor, vp, i64, vp]),
         "gemm_mxfp4_rmsnorm": (i32, [_Tensor, _Tensor, vp, i32, i64, f32, vp, i64, vp]),
         "gemm_mxfp4_swiglu": (i32, [_Tensor, _Tensor, vp, i64, ctypes.POINTER(_Tensor), vp]),
+        "nvfp4_signal_barrier": (i32, [vp, i32, i32, ctypes.c_uint32, i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -329,6 +330,18 @@ class FakeQuantizeSTE(torch.autograd.Function):
 
 def read_device_status(stream=None) -> int:
     return int(load().nvfp4_read_device_status(_stream(stream)))
+
+
+def signal_barrier(signal_ptrs: torch.Tensor, rank: int, epoch: int, limit_ns: int = 10_000_000_000,
+                   stream=None) -> None:
+    """Barrier over peer-mapped signal words: signal_ptrs is a device int64 tensor of the
+    world's signal-array addresses (see nvfp4_signal_barrier). A rank that does not arrive
+    within limit_ns ends this rank's wait with NVFP4_ERR_DEVICE_TIMEOUT in the device status
+    word (read_device_status) instead of holding the GPU."""
+    if signal_ptrs.dtype != torch.int64 or not signal_ptrs.is_cuda:
+        raise RuntimeError("signal_ptrs must be a CUDA int64 tensor of addresses")
+    _check(load().nvfp4_signal_barrier(signal_ptrs.data_ptr(), signal_ptrs.numel(), rank, epoch & 0xFFFFFFFF,
+                                       limit_ns, _stream(stream)), "nvfp4_signal_barrier")
 
 
 def selftest_bounded_wait(limit_ns: int, stream=None) -> None:

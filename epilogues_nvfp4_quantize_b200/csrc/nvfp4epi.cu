@@ -586,6 +586,64 @@ NVFP4_API nvfp4_status nvfp4_selftest_bounded_wait(int64_t limit_ns, cudaStream_
 NVFP4_API int64_t nvfp4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 // -------------------------------------------------------------------------------------
+// Stream-ordered barrier over peer-mapped signal words (one process per GPU), for the
+// row-parallel GEMM whose epilogue adds into the other ranks' output blocks.
+// -------------------------------------------------------------------------------------
+namespace {
+
+__device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Thread q < world publishes `epoch` in slot [rank] of rank q's signal words (after a
+// system-scope fence, so everything this GPU wrote before, the previous kernels' additions
+// into peer blocks included, is visible to q first), then waits until slot [q] of this
+// rank's words has reached `epoch`. A wait that runs past limit_ns records
+// NVFP4_ERR_DEVICE_TIMEOUT in the device status word and returns.
+__global__ void __launch_bounds__(64) signal_barrier_kernel(uint32_t* const* __restrict__ signals, int world,
+                                                            int rank, uint32_t epoch, uint64_t limit_ns) {
+  const int q = threadIdx.x;
+  if (q < world) {
+    __threadfence_system();
+    st_release_sys(signals[q] + rank, epoch);
+  }
+  __syncthreads();
+  if (q < world) {
+    const uint32_t* mine = signals[rank] + q;
+    const uint64_t t0 = nvfp4::globaltimer_ns();
+    while (static_cast<int32_t>(ld_acquire_sys(mine) - epoch) < 0) {
+      if (nvfp4::globaltimer_ns() - t0 > limit_ns) {
+        nvfp4::record_status(NVFP4_ERR_DEVICE_TIMEOUT, 70);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+}
+
+}  // namespace
+
+NVFP4_API nvfp4_status nvfp4_signal_barrier(uint32_t* const* signals, int world, int rank, uint32_t epoch,
+                                            int64_t limit_ns, cudaStream_t stream) {
+  if (signals == nullptr || epoch == 0) return NVFP4_ERR_INVALID_ARG;
+  if (world < 1 || world > 64 || rank < 0 || rank >= world) return NVFP4_ERR_INVALID_ARG;
+  if (limit_ns < 1 || limit_ns > 60000000000ll) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(signals) & 7u) != 0) return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceInfo* info;
+  nvfp4_status st;
+  if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
+  signal_barrier_kernel<<<1, 64, 0, stream>>>(signals, world, rank, epoch, static_cast<uint64_t>(limit_ns));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
+// -------------------------------------------------------------------------------------
 // Allocation-free quantiser: nvfp4_quantize with compute_amax = 1, whose scratch (one
 // partial maximum per block of 16384 input values, then the tensor's amax) lives in a
 // file-scope device array instead of a caller workspace.

@@ -15,13 +15,17 @@ touching the epilogues:
 - FFN-down, row-parallel: rank r multiplies its intermediate columns by the matching K
   slice of the down weight; the partial sums over the ranks are added up, leaving rank r
   the output rows [r M/w, (r+1) M/w). Two ways:
-  - reduce="nccl": the GEMM writes float32 partials (pointwise epilogue, f32 cast), then
+  - reduce="nccl": the GEMM writes its partials (pointwise epilogue: float32 by default, or
+    bf16 with partials="bf16", half the NVLink bytes at one bf16 rounding per rank), then
     one NCCL reduce-scatter over the token rows;
   - reduce="fused": the GEMM's epilogue adds each partial row straight into its owner's
     output block (gemm_nvfp4_reduce_rows_f32). The blocks are symmetric memory, so every
     rank holds the others' addresses. A barrier before the GEMM means every block is
-    zeroed; a barrier after it means every addition has landed. The only traffic between
-    GPUs is those stores: no kernel loads from another GPU's memory.
+    zeroed; a barrier after it means every addition has landed. The barrier is the
+    library's own kernel (nvfp4_signal_barrier) on peer-mapped signal words: its waits are
+    bounded, and a rank that never arrives ends the others' wait with a status in the
+    device status word, leaving their GPUs usable. The only traffic between GPUs is those
+    stores and signal words: no kernel loads data from another GPU's memory.
 
 The index helpers below are pure host logic (tested with gloo ranks on the CPU); TPLayer
 runs them with the library's kernels and NCCL or symmetric memory.
@@ -79,12 +83,14 @@ class TPLayer:
 
     Weights are given whole (bf16, on this rank's device) and sharded here; each rank
     packs only its shard. step(xq) takes the NVFP4 activations (replicated, M x K) and
-    returns (qkv_local bf16 M x 3*(heads/w)*head_dim, out_rows float32 (M/w) x K).
+    returns (qkv_local bf16 M x 3*(heads/w)*head_dim, out_rows (M/w) x K: float32, or bf16
+    with reduce="nccl", partials="bf16").
     With reduce="fused", out_rows is this rank's symmetric-memory block for that M: the next
     step of the same M zeroes and refills it, so copy it out to keep it."""
 
     def __init__(self, w_qkv, w_up, w_down, w_norm_q, w_norm_k, heads: int, head_dim: int,
-                 h_gscale: float, group=None, eps: float = 1e-6, reduce: str = "nccl"):
+                 h_gscale: float, group=None, eps: float = 1e-6, reduce: str = "nccl",
+                 partials: str = "f32"):
         import torch
         import torch.distributed as dist
         from . import _lib as L
@@ -113,7 +119,12 @@ class TPLayer:
         if reduce not in ("nccl", "fused"):
             raise ValueError(f"reduce must be 'nccl' or 'fused', not {reduce!r}")
         self.reduce = reduce
-        self._fused = {}  # M -> (this rank's output block, symmetric-memory handle or None, pointers)
+        if partials not in ("f32", "bf16"):
+            raise ValueError(f"partials must be 'f32' or 'bf16', not {partials!r}")
+        self.partial_dtype = torch.float32 if partials == "f32" else torch.bfloat16
+        self._fused = {}  # M -> (this rank's output block, signal-array pointers or None, block pointers)
+        self._epoch = 0   # barriers taken so far (the signal words count them)
+        self.barrier_limit_ns = 10_000_000_000
 
     def _pack(self, whole, shard, interleave: bool = False):
         T, L = self.L.NVFP4Tensor, self.L
@@ -134,15 +145,15 @@ class TPLayer:
         h.gscale.fill_(self.h_gscale)  # static scale, the same on every rank
         L.gemm_nvfp4_swiglu(xq, self.Wup, None, h)
         if self.reduce == "fused":
-            out, hdl, ptrs = self._fused_block(M, dev)
+            out, sig, ptrs = self._fused_block(M, dev)
             out.zero_()
-            self._barrier(hdl)  # every rank's block is zeroed before any rank adds into it
+            self._barrier(sig)  # every rank's block is zeroed before any rank adds into it
             L.gemm_nvfp4_reduce_rows_f32(h, self.Wdown, ptrs, M // self.world, self.Wdown.rows)
-            self._barrier(hdl)  # every rank's additions have landed
+            self._barrier(sig)  # every rank's additions have landed
             return qkv, out
-        part = torch.empty(M, self.Wdown.rows, dtype=torch.float32, device=dev)
+        part = torch.empty(M, self.Wdown.rows, dtype=self.partial_dtype, device=dev)
         L.gemm_nvfp4_pointwise(h, self.Wdown, part)
-        out = torch.empty(M // self.world, self.Wdown.rows, dtype=torch.float32, device=dev)
+        out = torch.empty(M // self.world, self.Wdown.rows, dtype=self.partial_dtype, device=dev)
         if self.world > 1:
             self.dist.reduce_scatter_tensor(out, part, group=self.group)
         else:
@@ -159,19 +170,30 @@ class TPLayer:
             n = self.Wdown.rows
             if self.world > 1:
                 import torch.distributed._symmetric_memory as symm_mem
+                group = self.group if self.group is not None else self.dist.group.WORLD
                 block = symm_mem.empty((rows.stop - rows.start, n), dtype=torch.float32, device=dev)
-                hdl = symm_mem.rendezvous(block, self.group if self.group is not None else self.dist.group.WORLD)
+                hdl = symm_mem.rendezvous(block, group)
                 ptrs = torch.tensor(list(hdl.buffer_ptrs), dtype=torch.int64, device=dev)
+                # one uint32 signal word per rank, in symmetric memory too, zeroed on every
+                # rank before any rank's first barrier
+                words = symm_mem.empty((self.world,), dtype=torch.int32, device=dev)
+                words.zero_()
+                shdl = symm_mem.rendezvous(words, group)
+                sig = (words, torch.tensor(list(shdl.buffer_ptrs), dtype=torch.int64, device=dev))
+                torch.cuda.synchronize(dev)
+                self.dist.barrier(group=self.group)
             else:
                 block = torch.empty(rows.stop - rows.start, n, dtype=torch.float32, device=dev)
-                hdl = None
+                sig = None
                 ptrs = torch.tensor([block.data_ptr()], dtype=torch.int64, device=dev)
-            self._fused[M] = (block, hdl, ptrs)
+            self._fused[M] = (block, sig, ptrs)
         return self._fused[M]
 
-    def _barrier(self, hdl):
-        """Stream-ordered barrier over the ranks' symmetric memory (nothing to wait for at
-        world size 1). Bounded: a rank that never arrives ends the wait after 10 s instead of
-        holding the others forever."""
-        if hdl is not None:
-            hdl.barrier(channel=0, timeout_ms=10_000)
+    def _barrier(self, sig):
+        """Stream-ordered barrier over the ranks' signal words (nothing to wait for at world
+        size 1): the library's bounded barrier kernel. A rank that never arrives ends the
+        others' wait after barrier_limit_ns with NVFP4_ERR_DEVICE_TIMEOUT in their device
+        status words; their kernels return and their contexts stay usable."""
+        if sig is not None:
+            self._epoch += 1
+            self.L.signal_barrier(sig[1], self.rank, self._epoch, self.barrier_limit_ns)

@@ -285,7 +285,9 @@ nvfp4_status swiglu_bf16(const void* c, int64_t rows, int64_t nh, int64_t ldc,
  *     NVFP4_ERR_UNSUPPORTED_SHAPE and nothing is launched; the other rules are those of
  *     nvfp4_quantize.
  *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
+ *     that device current); make that first call before any stream capture. The address is
+ *     kept for the life of the process: do not call this after a cudaDeviceReset of that
+ *     device in the same process.
  *   - All calls share the array and leave their values in it. Every value a call reads is
  *     written earlier by the same call, so nothing needs clearing, but calls whose kernels
  *     overlap on the GPU (different streams, or different host threads) race on the array
@@ -313,6 +315,26 @@ int nvfp4_read_device_status(cudaStream_t stream);
  * returns normally, leaving the context usable.
  */
 nvfp4_status nvfp4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream);
+
+/*
+ * Barrier of the tensor-parallel FFN-down reduction (the row-parallel GEMM whose epilogue
+ * adds its partial rows into the owners' blocks, gemm_nvfp4_reduce_rows_f32; page "Serving
+ * sub-second Ideogram v4 without quality loss", section "Epilogue fusion in brief": output
+ * tiles are independent, so only this reduction crosses GPUs). One process per GPU; every
+ * rank launches it on its stream with the same `epoch`.
+ *   signals: device array of `world` pointers; signals[q] is rank q's array of `world`
+ *            uint32 words (peer-mapped, e.g. symmetric memory), zeroed once before the
+ *            first barrier. signals[rank] is this rank's own array.
+ *   epoch:   1, 2, 3, ... one more per barrier (0 is invalid); wraps modulo 2^32.
+ * The kernel fences at system scope, writes `epoch` into word [rank] of every rank's
+ * array, then waits until every word of its own array has reached `epoch`. A wait longer
+ * than limit_ns nanoseconds (1 .. 6e10) gives up: NVFP4_ERR_DEVICE_TIMEOUT is recorded in
+ * the device status word (nvfp4_read_device_status) and the kernel returns, leaving the
+ * context usable. Argument errors return NVFP4_ERR_INVALID_ARG (or MISALIGNED for an
+ * unaligned pointer array) and launch nothing.
+ */
+nvfp4_status nvfp4_signal_barrier(uint32_t* const* signals, int world, int rank, uint32_t epoch,
+                                  int64_t limit_ns, cudaStream_t stream);
 
 /* Number of kernels the library has launched in this process (for launch accounting). */
 int64_t nvfp4_launch_count(void);

@@ -90,6 +90,13 @@ def test_argument_checks_return_status_without_gpu(lib):
     assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 1, 128, 256, None) == SHAPE  # M != w*rows
     assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 2, 128, 200, None) == INVALID  # ldd < N
     assert lib.gemm_nvfp4_reduce_rows_f32(_t(256, 256), _t(256, 256), 16, 2, 128, 258, None) == MISALIGNED
+    # signal barrier: pointer array, world, rank, epoch, limit
+    assert lib.nvfp4_signal_barrier(None, 2, 0, 1, 1000, None) == INVALID
+    assert lib.nvfp4_signal_barrier(16, 0, 0, 1, 1000, None) == INVALID      # world < 1
+    assert lib.nvfp4_signal_barrier(16, 2, 2, 1, 1000, None) == INVALID      # rank >= world
+    assert lib.nvfp4_signal_barrier(16, 2, 0, 0, 1000, None) == INVALID      # epoch 0
+    assert lib.nvfp4_signal_barrier(16, 2, 0, 1, 0, None) == INVALID         # limit 0
+    assert lib.nvfp4_signal_barrier(12, 2, 0, 1, 1000, None) == MISALIGNED   # array % 8
 
 
 def test_empty_inputs_are_rejected_before_any_launch(lib):

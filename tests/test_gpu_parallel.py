@@ -59,3 +59,42 @@ def test_tp_layer_world1_equals_the_unsharded_kernels(M, reduce):
     qd, sd, gd = o.quantized_operand(wdc)
     out_o = o.gemm(o.dequantize(qh, sh, np.float32(G_h)), o.dequantize(qd, sd, gd))
     assert_close(out.cpu().numpy().astype(np.float64), out_o, "TPLayer FFN vs oracle")
+
+
+def test_tp_layer_bf16_partials_world1_matches_the_oracle():
+    dev = device()
+    M, heads, hd, K, nh = 256, 4, 128, 512, 512
+    x = wk.activations(M, K, 1, seed=9).to(dev)
+    wq = wk.weights(3 * heads * hd, K, 1 / np.sqrt(K), seed=1).to(dev)
+    wu = wk.weights(2 * nh, K, 1 / np.sqrt(K), seed=2).to(dev)
+    wd = wk.weights(K, nh, 1 / np.sqrt(nh), seed=3).to(dev)
+    wn = torch.from_numpy(wk.norm_weight(hd, 0, 3)).to(dev)
+    xq = ep.nvfp4_quantize(x, ep.NVFP4Tensor.empty(M, K, dev))
+    G_h = 0.01
+    layer = TPLayer(wq, wu, wd, wn, wn, heads, hd, G_h, reduce="nccl", partials="bf16")
+    _, out = layer.step(xq)
+    assert out.dtype == torch.bfloat16
+    h_o = o.problem_swiglu(x.cpu(), wu.cpu())
+    qh, sh, _ = o.requantize(h_o, np.float32(G_h))
+    qd, sd, gd = o.quantized_operand(wd.cpu())
+    out_o = o.bf16_round(o.gemm(o.dequantize(qh, sh, np.float32(G_h)), o.dequantize(qd, sd, gd)))
+    assert_close(out.float().cpu().numpy().astype(np.float64), out_o, "TPLayer bf16 partials vs oracle")
+
+
+def test_signal_barrier_passes_alone_and_times_out_into_a_status():
+    """World size 1: the barrier waits only for its own word and passes. Then a two-rank
+    barrier whose second rank does not exist: this rank's wait on a word that nothing sets
+    runs out after 2 ms, records NVFP4_ERR_DEVICE_TIMEOUT and returns; the context stays
+    usable."""
+    dev = device()
+    assert ep.read_device_status() == 0
+    own = torch.zeros(2, dtype=torch.int32, device=dev)
+    ep.signal_barrier(torch.tensor([own.data_ptr()], dtype=torch.int64, device=dev), 0, 1)
+    assert ep.read_device_status() == 0
+    assert own[0].item() == 1
+    other = torch.zeros(2, dtype=torch.int32, device=dev)
+    ptrs = torch.tensor([own.data_ptr(), other.data_ptr()], dtype=torch.int64, device=dev)
+    ep.signal_barrier(ptrs, 0, 2, limit_ns=2_000_000)
+    assert ep.read_device_status() == 6
+    assert own[0].item() == 2 and other[0].item() == 2 and own[1].item() == 0
+    assert ep.read_device_status() == 0
