@@ -657,9 +657,9 @@ class OracleLayer:
         self.x = wk.activations(M, K_IN, wk.outlier_count(K_IN), seed=seed).float().numpy()
         std = 1.0 / np.sqrt(K_IN)
         t0 = time.perf_counter()
-        self.Bqkv = o.dequantize(*o.quantize(wk.weights(N_QKV, K_IN, std, seed=seed, stream=11).float().numpy()))
-        self.Bup = o.dequantize(*o.quantize(wk.weights(N_UP, K_IN, std, seed=seed, stream=12).float().numpy()))
-        self.Bdown = o.dequantize(*o.quantize(
+        self.Bqkv = o.dequantize(*o.quantize_fp32_order(wk.weights(N_QKV, K_IN, std, seed=seed, stream=11).float().numpy()))
+        self.Bup = o.dequantize(*o.quantize_fp32_order(wk.weights(N_UP, K_IN, std, seed=seed, stream=12).float().numpy()))
+        self.Bdown = o.dequantize(*o.quantize_fp32_order(
             wk.weights(K_IN, K_DOWN, 1.0 / np.sqrt(K_DOWN), seed=seed, stream=13).float().numpy()))
         self.pack_s = time.perf_counter() - t0
         wq, wkk = wk.norm_weight(HD, seed, 3), wk.norm_weight(HD, seed, 5)
@@ -670,7 +670,7 @@ class OracleLayer:
     def step(self, rows):
         o = self.o
         xs = self.x[rows]
-        qa, sa, _ = o.quantize(xs, self.Gx)
+        qa, sa, _ = o.quantize_fp32_order(xs, self.Gx)
         a = o.dequantize(qa, sa, self.Gx)
         qkv = o.bf16_round(o.rmsnorm_heads(o.gemm(a, self.Bqkv), self.w, HD, N_NORM, EPS))
         h = o.bf16_round(o.swiglu(o.gemm(a, self.Bup)))

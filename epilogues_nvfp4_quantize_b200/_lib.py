@@ -130,13 +130,24 @@ def quantize_workspace_bytes() -> int:
     return int(load().nvfp4_quantize_workspace_bytes())
 
 
+def _workspace(workspace: Optional[torch.Tensor], compute_amax: bool, device) -> Optional[torch.Tensor]:
+    """The caller's workspace (checked for size), or a new one when none is given."""
+    if not compute_amax:
+        return workspace
+    need = quantize_workspace_bytes()
+    if workspace is None:
+        return torch.empty((need,), dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace holds {workspace.numel() * workspace.element_size()} bytes, needs {need}")
+    return workspace
+
+
 def nvfp4_quantize(x: torch.Tensor, out: NVFP4Tensor, compute_amax: bool = True, interleave: bool = False,
                    workspace: Optional[torch.Tensor] = None, stream=None) -> NVFP4Tensor:
     """Quantise a bf16 2-D CUDA tensor into `out` (see nvfp4_quantize in the header)."""
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be a 2-D bf16 tensor with unit column stride")
-    if compute_amax and workspace is None:
-        workspace = torch.empty((quantize_workspace_bytes(),), dtype=torch.uint8, device=x.device)
+    workspace = _workspace(workspace, compute_amax, x.device)
     _check(load().nvfp4_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), int(compute_amax),
                                  SWIGLU_INTERLEAVE if interleave else 0, out.c(), _ptr(workspace),
                                  _stream(stream)), "nvfp4_quantize")
@@ -306,8 +317,7 @@ def nvfp4_fake_quantize(x: torch.Tensor, y: Optional[torch.Tensor] = None, gscal
         if not compute_amax:
             raise ValueError("a static scale needs gscale")
         gscale = torch.empty((1,), dtype=torch.float32, device=x.device)
-    if compute_amax and workspace is None:
-        workspace = torch.empty((quantize_workspace_bytes(),), dtype=torch.uint8, device=x.device)
+    workspace = _workspace(workspace, compute_amax, x.device)
     _check(load().nvfp4_fake_quantize(x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), int(compute_amax),
                                       gscale.data_ptr(), py, ldy, _ptr(workspace), _stream(stream)),
            "nvfp4_fake_quantize")

@@ -301,12 +301,82 @@ static nvfp4_status launch_quantize_stream(DeviceInfo* info, const void* x, int6
   return launch_status();
 }
 
+// Launch of the two-kernel quantiser (quantize.cuh) for nvfp4_quantize and
+// nvfp4_fake_quantize: with compute_amax, the amax partials kernel then the quantise kernel
+// (programmatic dependent launch); with a static scale, the quantise kernel alone.
+static nvfp4_status launch_quantize2(DeviceInfo* info, const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                     int compute_amax, bool inter, float* gscale, uint8_t* codes, uint8_t* sf,
+                                     uint16_t* y, int64_t ldy, void* workspace, cudaStream_t stream) {
+  using namespace nvfp4::q2cfg;
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  // 256-bit accesses need every row of x (and of y) to start on a 32-byte boundary
+  const bool x_v8 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  const bool y_v8 = y == nullptr || ((reinterpret_cast<uintptr_t>(y) & 31u) == 0 && (ldy % 16) == 0);
+  nvfp4::Quant2Args qa{};
+  qa.x = xp;
+  qa.rows = rows;
+  qa.cols = cols;
+  qa.ldx = ldx;
+  qa.interleave = inter ? 1 : 0;
+  qa.gscale = gscale;
+  qa.codes = codes;
+  qa.sf = sf;
+  qa.y = y;
+  qa.ldy = ldy;
+  if (compute_amax) {
+    const int64_t chunks = rows * (cols / 16);
+    int64_t parts = (chunks + 4 * AMAX_THREADS - 1) / (4 * AMAX_THREADS);
+    const int64_t cap = 2ll * info->sm_count < MAX_PARTIALS ? 2ll * info->sm_count : MAX_PARTIALS;
+    if (parts > cap) parts = cap;
+    if (parts < 1) parts = 1;
+    float* partials = static_cast<float*>(workspace);
+    const dim3 grid(static_cast<unsigned>(parts));
+    if (ldx == cols && x_v8) {
+      nvfp4::amax_partial_kernel<true, true><<<grid, AMAX_THREADS, 0, stream>>>(xp, rows, cols, ldx, partials);
+    } else if (ldx == cols) {
+      nvfp4::amax_partial_kernel<true, false><<<grid, AMAX_THREADS, 0, stream>>>(xp, rows, cols, ldx, partials);
+    } else if (x_v8) {
+      nvfp4::amax_partial_kernel<false, true><<<grid, AMAX_THREADS, 0, stream>>>(xp, rows, cols, ldx, partials);
+    } else {
+      nvfp4::amax_partial_kernel<false, false><<<grid, AMAX_THREADS, 0, stream>>>(xp, rows, cols, ldx, partials);
+    }
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    nvfp4_status st;
+    if ((st = launch_status()) != NVFP4_OK) return st;
+    qa.partials = partials;
+    qa.nparts = static_cast<int>(parts);
+  }
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  const int64_t tasks = rows_pad * ((cols / 64 + 7) / 8);
+  int64_t grid = (tasks + QUANT_WARPS - 1) / QUANT_WARPS;
+  const int64_t full = 8ll * info->sm_count;  // 8 CTAs of 256 threads fill an SM
+  if (grid > full) grid = full;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(QUANT_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = (x_v8 && y_v8) ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<true>, qa)
+                                       : cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<false>, qa);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return launch_status();
+}
+
 NVFP4_API int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols) {
   if (rows < 0 || cols < 0) return -1;
   return ((rows + 127) / 128) * 128 * ((cols / 16 + 3) / 4) * 4;
 }
 
-NVFP4_API int64_t nvfp4_quantize_workspace_bytes(void) { return 16; }
+NVFP4_API int64_t nvfp4_quantize_workspace_bytes(void) {
+  return nvfp4::q2cfg::MAX_PARTIALS * static_cast<int64_t>(sizeof(float));
+}
 
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int compute_amax,
                                       int flags, nvfp4_tensor out, void* workspace, cudaStream_t stream) {
@@ -328,9 +398,9 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t cols,
   nvfp4_status st;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
 
-  return launch_quantize_stream(info, x, rows, cols, ldx, compute_amax, (flags & NVFP4_SWIGLU_INTERLEAVE) != 0,
-                                out.gscale, static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf), nullptr,
-                                0, workspace, stream);
+  return launch_quantize2(info, x, rows, cols, ldx, compute_amax, (flags & NVFP4_SWIGLU_INTERLEAVE) != 0,
+                          out.gscale, static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf), nullptr, 0,
+                          workspace, stream);
 }
 
 NVFP4_API nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t cols, int64_t ldx, int compute_amax,
@@ -349,8 +419,8 @@ NVFP4_API nvfp4_status nvfp4_fake_quantize(const void* x, int64_t rows, int64_t 
   DeviceInfo* info;
   nvfp4_status st;
   if ((st = current_device(&dev, &info)) != NVFP4_OK) return st;
-  return launch_quantize_stream(info, x, rows, cols, ldx, compute_amax, false, gscale, nullptr, nullptr,
-                                static_cast<uint16_t*>(y), ldy, workspace, stream);
+  return launch_quantize2(info, x, rows, cols, ldx, compute_amax, false, gscale, nullptr, nullptr,
+                          static_cast<uint16_t*>(y), ldy, workspace, stream);
 }
 
 NVFP4_API nvfp4_status gemm_nvfp4_plain(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t ldd,

@@ -381,6 +381,212 @@ __global__ void __launch_bounds__(qcfg::THREADS, 1)
 }
 
 // =====================================================================================
+// Two-kernel quantiser (the path of nvfp4_quantize and nvfp4_fake_quantize).
+//
+// 1. amax_partial_kernel streams x once (HBM-bound) and writes one partial max|x| per CTA
+//    into the caller's workspace. Its loads ask L2 to keep x.
+// 2. quantize_rows_kernel is launched with programmatic dependent launch: its CTAs may
+//    become resident while the first kernel drains, and wait (griddepcontrol.wait) until
+//    that kernel's partials are visible. Each CTA reduces the partials to the tensor's amax,
+//    derives G = amax / (6 * 448), and fills a shared table of the 127 block-scale
+//    reciprocals 1 / (e4m3(s) * G). Then every lane quantises one 16-value block: one
+//    32-byte load (a warp reads 1 KB of a row), the block's E4M3 scale, one table lookup
+//    for the reciprocal, 16 products and 8 E2M1 conversions, an 8-byte code store; lanes
+//    4k..4k+3 are the 4 blocks of one scale word, assembled with two shuffles. Row tasks
+//    run in the reverse order of the first kernel's reads, so the data read last (likeliest
+//    still in L2) is quantised first.
+// No grid barrier and no workspace clearing: every partial a call reads is written by the
+// same call.
+// =====================================================================================
+namespace q2cfg {
+constexpr int AMAX_THREADS = 512;
+constexpr int QUANT_THREADS = 256;
+constexpr int QUANT_WARPS = QUANT_THREADS / 32;
+constexpr int MAX_PARTIALS = 1024;  // floats of workspace: one per CTA of the amax kernel
+}  // namespace q2cfg
+
+// 32 bytes (16 bf16) from global memory with an L2 eviction policy: one 256-bit access when
+// the address is 32-byte aligned (V8), else two 128-bit accesses (16-byte aligned).
+template <bool V8>
+__device__ __forceinline__ void ld_global_32b(const void* p, uint64_t policy, uint32_t (&w)[8]) {
+  if constexpr (V8) {
+    asm("ld.global.nc.L2::cache_hint.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
+        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+        : "l"(p), "l"(policy));
+  } else {
+    const char* c = static_cast<const char*>(p);
+    asm("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+        : "l"(c), "l"(policy));
+    asm("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+        : "l"(c + 16), "l"(policy));
+  }
+}
+template <bool V8>
+__device__ __forceinline__ void st_global_32b(void* p, const uint32_t (&w)[8]) {
+  if constexpr (V8) {
+    asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  } else {
+    uint4* q = static_cast<uint4*>(p);
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+// Programmatic dependent launch: let the next kernel in the stream start launching, and
+// wait until the previous kernel has completed with its memory visible (a no-op when this
+// kernel was launched without the programmatic attribute).
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Block-wide maximum of a non-negative float (blockDim.x a multiple of 32, at most 1024).
+__device__ __forceinline__ float block_max(float m, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  if (warp == 0) {
+    m = lane < static_cast<int>(blockDim.x >> 5) ? s_red[lane] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  }
+  return m;  // valid in warp 0
+}
+
+// One partial max|x| per CTA over rows x cols bf16 (row pitch ldx, cols % 64 == 0), viewed
+// as 32-byte chunks: consecutive threads read consecutive chunks, four chunks in flight.
+template <bool CONTIG, bool V8>
+__global__ void __launch_bounds__(q2cfg::AMAX_THREADS, CONTIG ? 2 : 1) amax_partial_kernel(const uint16_t* __restrict__ x,
+                                                                           int64_t rows, int64_t cols, int64_t ldx,
+                                                                           float* __restrict__ partial) {
+  __shared__ float s_red[32];
+  griddep_launch_dependents();  // the quantise kernel waits for this grid's completion anyway
+  const uint64_t keep = l2_policy_evict_last();
+  const int64_t cpr = cols >> 4;  // 32-byte chunks per row
+  const int64_t total = rows * cpr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  auto addr = [&](int64_t c) -> const uint16_t* {
+    if constexpr (CONTIG) {
+      return x + c * 16;
+    } else {
+      const int64_t r = c / cpr;
+      return x + r * ldx + (c - r * cpr) * 16;
+    }
+  };
+  uint32_t m = 0u;  // packed |bf16| maxima (max.xorsign.abs leaves a sign that is dropped below)
+  int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; c + 3 * stride < total; c += 4 * stride) {
+    uint32_t w[4][8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ld_global_32b<V8>(addr(c + k * stride), keep, w[k]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[k][j]));
+  }
+  for (; c < total; c += stride) {
+    uint32_t w[8];
+    ld_global_32b<V8>(addr(c), keep, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[j]));
+  }
+  const float f = fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
+  const float b = block_max(f, s_red);
+  if (threadIdx.x == 0) partial[blockIdx.x] = b;
+}
+
+struct Quant2Args {
+  const uint16_t* x;
+  int64_t rows, cols, ldx;  // output rows (after the optional interleave) and columns
+  int interleave;           // output row 2j <- input row j, 2j+1 <- input row rows/2 + j
+  const float* partials;    // amax partials of the first kernel (null: static *gscale)
+  int nparts;
+  float* gscale;
+  uint8_t* codes;           // codes and scales (or null: fake quantisation only)
+  uint8_t* sf;
+  uint16_t* y;              // quantise-dequantise output in bf16 (or null)
+  int64_t ldy;
+};
+
+// V8: x (and y) rows start on 32-byte boundaries, so each lane's 16 values move in one
+// 256-bit access.
+template <bool V8>
+__global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(const Quant2Args a) {
+  using namespace q2cfg;
+  __shared__ float s_rcp[128];
+  __shared__ float s_red[32];
+  __shared__ float s_G;
+  griddep_wait();  // the amax partials (or the producer of x) are complete and visible
+  if (a.partials != nullptr) {
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < a.nparts; i += blockDim.x) m = fmaxf(m, a.partials[i]);
+    m = block_max(m, s_red);
+    if (threadIdx.x == 0) {
+      const float g = __fdiv_rn(m, kGlobalDiv);
+      s_G = g;
+      if (blockIdx.x == 0) *a.gscale = g;
+    }
+  } else if (threadIdx.x == 0) {
+    s_G = *a.gscale;
+  }
+  __syncthreads();
+  const float G = s_G;
+  const float enc = scale_encode_factor(G);
+  // reciprocal of every block scale d = e4m3(s) * G (0 where d is 0; code 0x7F is NaN and
+  // never produced by the saturating conversion)
+  if (threadIdx.x < 128) s_rcp[threadIdx.x] = threadIdx.x == 0x7F ? 0.0f : block_inv_scale(threadIdx.x, G);
+  __syncthreads();
+
+  const uint64_t stream = l2_policy_evict_first();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane & 3;                       // block of the lane's 64-value group
+  const int64_t ng = a.cols >> 6;                 // 64-value groups (scale words) per row
+  const int64_t tpr = (ng + 7) >> 3;              // warp tasks per row: 8 groups each
+  const int64_t rows_pad = (a.rows + 127) & ~int64_t(127);
+  const int64_t tasks = rows_pad * tpr;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * QUANT_WARPS;
+  for (int64_t t = tasks - 1 - (static_cast<int64_t>(blockIdx.x) * QUANT_WARPS + warp); t >= 0; t -= nwarps) {
+    const int64_t row = t / tpr;
+    const int64_t g = (t - row * tpr) * 8 + (lane >> 2);
+    const bool live = g < ng && row < a.rows;
+    uint32_t s = 0u;
+    if (live) {
+      const int64_t src = a.interleave ? ((row & 1) ? (a.rows >> 1) + (row >> 1) : (row >> 1)) : row;
+      uint32_t w[8];
+      ld_global_32b<V8>(a.x + src * a.ldx + g * 64 + sub * 16, stream, w);
+      s = block_scale_code(bf16x16_amax(w), enc);
+      const float r = s_rcp[s];
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[2 * j] = bf16_lo(w[j]);
+        v[2 * j + 1] = bf16_hi(w[j]);
+      }
+      uint32_t lo = block_codes8(v, r), hi = block_codes8(v + 8, r);
+      if (!(r > 0.0f)) lo = hi = 0u;  // d == 0: every code of the block is 0
+      if (a.codes != nullptr) {
+        *reinterpret_cast<uint2*>(a.codes + row * (a.cols >> 1) + g * 32 + sub * 8) = make_uint2(lo, hi);
+      }
+      if (a.y != nullptr) {
+        uint32_t o[8];
+        dequant_block16_bf16(lo, hi, s, G, o);
+        st_global_32b<V8>(a.y + row * a.ldy + g * 64 + sub * 16, o);
+      }
+    }
+    // the scale word of each 64-value group: byte `sub` from lane 4k + sub (0 for padding rows)
+    uint32_t word = s << (8 * sub);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if (a.codes != nullptr && sub == 0 && g < ng) {
+      *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(row, 4 * g, a.cols >> 4)) = word;
+    }
+  }
+}
+
+// =====================================================================================
 // MXFP4 (OCP Microscaling: E2M1 elements, one E8M0 scale per 32) with an optional fixed
 // block-local transform, the 32-point Walsh-Hadamard matrix H_2 (x) ... (x) H_2 (page
 // "KroQuant: efficient post-training quantization for diffusion transformers via

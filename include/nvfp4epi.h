@@ -83,19 +83,28 @@ int64_t nvfp4_quantize_workspace_bytes(void);
 #define NVFP4_SWIGLU_INTERLEAVE 1
 
 /*
+ * Activation and weight quantisation ("Serving sub-second Ideogram v4 without quality
+ * loss", section "Running the transformer in FP4": E2M1 values; section
+ * "Quantization-aware distillation": dynamic or static per-tensor scales).
  * Quantise a bf16 tensor x (rows x cols, leading dimension ldx elements) to NVFP4.
  *   compute_amax = 1: G = amax(|x|) / (6 * 448) is computed on the device and written to
  *                     *out.gscale; `workspace` must hold
  *                     nvfp4_quantize_workspace_bytes() bytes, 4-byte aligned (contents on
- *                     entry ignored: the call clears it on `stream`). It holds the amax and
- *                     the counter of a grid barrier, so calls that share a workspace must
- *                     not overlap. The kernel is a cooperative launch (one CTA per SM); it
- *                     reads x twice, the second time mostly from L2.
+ *                     entry ignored: every value the call reads it writes first). It holds
+ *                     one partial amax per CTA of the first of two kernels; calls that
+ *                     share a workspace must not overlap on the GPU. The first kernel reads
+ *                     x once for its amax (asking L2 to keep it); the second, launched with
+ *                     programmatic dependent launch, reduces the partials and quantises,
+ *                     reading x again, mostly from L2. x rows that start on 32-byte
+ *                     boundaries are read with 256-bit accesses.
  *   compute_amax = 0: *out.gscale is used as given (static scale, must be > 0 and finite);
  *                     workspace may be NULL.
  * Per block of 16, in IEEE float32: s = E4M3_rn_satfinite(amax_b * (1 / (6 G))) (s = 0
  * for an all-zero block), d = e4m3(s) * G, q_i = E2M1_rn_satfinite(x_i * (1 / d)) (q = 0
- * when d = 0).
+ * when d = 0). These are the decisions of the plain rule (the E4M3 value nearest to
+ * amax_b / (6 G), the E2M1 value nearest to x_i / d, ties to even) except where an exact
+ * quotient lies within about 2^-21 (relative) of a rounding midpoint: at such a tie the
+ * float32 quotient may fall on either side, and either neighbouring code is correct.
  * flags: 0, or NVFP4_SWIGLU_INTERLEAVE: x is a [gate | up] weight of 2*Nh rows and output
  *        row 2j takes input row j, row 2j+1 takes input row Nh + j.
  * Rules: rows >= 1 (even with the interleave flag), cols % 64 == 0, ldx >= cols,
@@ -169,6 +178,9 @@ nvfp4_status gemm_mxfp4_swiglu(nvfp4_tensor A, nvfp4_tensor B, void* D, int64_t 
                                const nvfp4_tensor* Dq, cudaStream_t stream);
 
 /*
+ * Plain epilogue ("Serving sub-second Ideogram v4 without quality loss", section "Epilogue
+ * fusion in brief": the accumulator tile is scaled and written once; section "Running the
+ * transformer in FP4": the operands stay in 4 bits through the tensor-core MMA).
  * D (M x N bf16, leading dimension ldd) = bf16(G_A * G_B * sum_k A[m,k] * B[n,k]) with
  * A (M x K) and B (N x K) NVFP4, both K-contiguous.
  * Rules: M % 128 == 0, N % 256 == 0, K % 256 == 0, A.cols == B.cols == K,
@@ -229,6 +241,10 @@ nvfp4_status gemm_nvfp4_reduce_rows_f32(nvfp4_tensor A, nvfp4_tensor B, float* c
                                         int64_t rows_per_rank, int64_t ldd, cudaStream_t stream);
 
 /*
+ * Per-head RMSNorm epilogue ("Serving sub-second Ideogram v4 without quality loss",
+ * sections "Epilogue fusion in brief" (the formula), "Tiles and fragments on Blackwell" and
+ * "Why head_dim=256 is hard" (a head's sum of squares spans more than one thread's
+ * fragment), "Revisit fusion").
  * As gemm_nvfp4_plain, then per row and per head of head_dim adjacent columns among the
  * first n_norm_cols: y = x * rsqrt(mean(x^2) + eps) * w[col] (x = G_A G_B acc, float32);
  * columns >= n_norm_cols pass through (the V block of a QKV projection).
@@ -242,8 +258,11 @@ nvfp4_status gemm_nvfp4_rmsnorm(nvfp4_tensor A, nvfp4_tensor B, const float* w,
                                 void* D, int64_t ldd, cudaStream_t stream);
 
 /*
- * SwiGLU epilogue. B is the gate|up weight (N = 2*Nh rows) packed with
- * NVFP4_SWIGLU_INTERLEAVE, so accumulator columns come as [g0, u0, g1, u1, ...].
+ * SwiGLU epilogue ("Serving sub-second Ideogram v4 without quality loss", section "Fusing
+ * gated SiLU (SwiGLU)": gate = first half of the weight's rows, gate/up rows interleaved
+ * at packing time so each thread holds both; section "Quantization-aware distillation":
+ * the optional NVFP4 output uses a static scale). B is the gate|up weight (N = 2*Nh rows)
+ * packed with NVFP4_SWIGLU_INTERLEAVE, so accumulator columns come as [g0, u0, g1, u1, ...].
  *   out[m, j] = silu(x_g) * x_u, silu(x) = x / (1 + exp(-x)), x = G_A G_B acc.
  *   D  : M x Nh bf16 output (leading dimension ldd), or NULL.
  *   Dq : M x Nh NVFP4 output quantised from the bf16-rounded values with the static

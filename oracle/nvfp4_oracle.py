@@ -509,8 +509,16 @@ def _as_f32(t) -> np.ndarray:
 
 
 def quantized_operand(x_bf16):
-    """Quantise a bf16 operand with its own amax-derived G. Returns (codes, scales, G)."""
-    return quantize(_as_f32(x_bf16))
+    """Quantise a bf16 GEMM operand with its own amax-derived G. Returns (codes, scales, G).
+
+    The whole-problem functions below quantise their operands with the decisions taken in
+    float32 (``quantize_fp32_order``), the precision the kernels take them in. Where that
+    differs from the plain definition it is at a tie, where both results are correct, but
+    a GEMM needs one fixed choice: a block scale on the other side of a tie moves all 16
+    decoded values of the block by up to one scale step (12.5 %), and with the outlier
+    channels such blocks shift some outputs by more than the bf16 tolerance. The
+    quantiser itself is compared with the plain definition, tie rule included."""
+    return quantize_fp32_order(_as_f32(x_bf16))
 
 
 def problem_gemm(a_bf16, b_bf16, rows=None, b_quant=None) -> np.ndarray:
@@ -525,7 +533,7 @@ def problem_gemm(a_bf16, b_bf16, rows=None, b_quant=None) -> np.ndarray:
     Ga = global_scale(a)
     if rows is not None:
         a = a[np.asarray(rows)]
-    qa, sa, _ = quantize(a, Ga)
+    qa, sa, _ = quantize_fp32_order(a, Ga)
     qb, sb, gb = quantized_operand(b_bf16) if b_quant is None else b_quant
     return gemm(dequantize(qa, sa, Ga), dequantize(qb, sb, gb))
 
@@ -549,8 +557,10 @@ def problem_swiglu(a_bf16, b_gate_up_bf16, rows=None, b_quant=None) -> np.ndarra
 
 
 def requantize(out_bf16_values, G):
-    """Static-scale NVFP4 quantisation of bf16-valued outputs (blocks along N)."""
-    return quantize(np.asarray(out_bf16_values, np.float64).astype(F32), G)
+    """Static-scale NVFP4 quantisation of bf16-valued outputs (blocks along N), the decisions
+    taken in float32 like the operands of the whole-problem functions (the next GEMM's
+    input)."""
+    return quantize_fp32_order(np.asarray(out_bf16_values, np.float64).astype(F32), G)
 
 
 # ----------------------------------------------------------------------------------
