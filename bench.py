@@ -627,10 +627,16 @@ def run_cuda(args):
         ol = OracleLayer(M)
         ol.Gh = np.float32(layer.h.gscale.item())
         qkv_o, out_o = ol.step(check_rows)
-        e_qkv, e_out = max_rel_err(last_qkv, qkv_o), max_rel_err(last_out, out_o)
-        result["oracle_check"] = {"rows": len(check_rows), "qkv_max_rel": round(e_qkv, 5),
-                                  "out_max_rel": round(e_out, 5), "tolerance": 2e-2,
-                                  "ok": bool(e_qkv <= 2e-2 and e_out <= 2e-2)}
+        e_qkv = max_rel_err(last_qkv, qkv_o)
+        # the FFN-down output comes from re-quantised activations, whose codes may differ
+        # from the oracle's where the bf16 inputs differ: judged per element against
+        # 2e-2 |o| + 2e-2 rms(o), and normwise
+        rms_o = float(np.sqrt(np.mean(out_o * out_o)))
+        out_over = int(np.sum(np.abs(last_out - out_o) > 2e-2 * np.abs(out_o) + 2e-2 * rms_o))
+        out_norm = float(np.linalg.norm(last_out - out_o) / max(np.linalg.norm(out_o), 1e-300))
+        result["oracle_check"] = {"rows": len(check_rows), "qkv_max_rel": round(e_qkv, 5), "qkv_tolerance": 2e-2,
+                                  "out_elements_over": out_over, "out_normwise": round(out_norm, 6),
+                                  "ok": bool(e_qkv <= 2e-2 and out_over == 0 and out_norm <= 1e-3)}
         result["cpu_baseline"] = cpu_baseline(M, rows=args.cpu_rows, layer=ol)
 
     if world > 1:

@@ -36,6 +36,7 @@ struct DeviceInfo {
   bool pair_attr_set[2 * kEpiKinds] = {};
   int pair_clusters[2 * kEpiKinds] = {};
   bool quant_attr_set = false;
+  int quant_ctas_per_sm[2] = {0, 0};  // resident CTAs of quantize_rows_kernel<V8 = false, true>
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -346,10 +347,26 @@ static nvfp4_status launch_quantize2(DeviceInfo* info, const void* x, int64_t ro
     qa.partials = partials;
     qa.nparts = static_cast<int>(parts);
   }
+  const bool v8 = x_v8 && y_v8;
+  {
+    // CTAs that fit on an SM at once: the kernel's warps stride over the whole tensor, so a
+    // grid larger than one wave would only queue CTAs behind it
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int& per_sm = info->quant_ctas_per_sm[v8 ? 1 : 0];
+    if (per_sm == 0) {
+      int n = 0;
+      const cudaError_t e = v8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_rows_kernel<true>,
+                                                                               QUANT_THREADS, 0)
+                               : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_rows_kernel<false>,
+                                                                               QUANT_THREADS, 0);
+      if (e != cudaSuccess || n < 1) return NVFP4_ERR_CUDA;
+      per_sm = n;
+    }
+  }
   const int64_t rows_pad = (rows + 127) / 128 * 128;
   const int64_t tasks = rows_pad * ((cols / 64 + 7) / 8);
   int64_t grid = (tasks + QUANT_WARPS - 1) / QUANT_WARPS;
-  const int64_t full = 8ll * info->sm_count;  // 8 CTAs of 256 threads fill an SM
+  const int64_t full = static_cast<int64_t>(info->quant_ctas_per_sm[v8 ? 1 : 0]) * info->sm_count;
   if (grid > full) grid = full;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -362,8 +379,8 @@ static nvfp4_status launch_quantize2(DeviceInfo* info, const void* x, int64_t ro
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = (x_v8 && y_v8) ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<true>, qa)
-                                       : cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<false>, qa);
+  const cudaError_t e = v8 ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<true>, qa)
+                           : cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<false>, qa);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();

@@ -511,8 +511,43 @@ struct Quant2Args {
   int64_t ldy;
 };
 
+// E2M1 codes of 8 bf16 values (4 packed words) times r: the float32 products are formed two
+// at a time (mul.rn.f32x2, each product rounded like a scalar multiply).
+__device__ __forceinline__ uint32_t bf16x8_codes(const uint32_t* w, float r) {
+  float y[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %4};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(y[2 * j]), "=f"(y[2 * j + 1])
+        : "f"(bf16_lo(w[j])), "f"(bf16_hi(w[j])), "f"(r));
+  }
+  return cvt_e2m1x8(y);
+}
+
+// Quantise this lane's 16-value block (8 packed bf16 words): its scale code, 8 bytes of codes
+// (0 when the decoded scale is 0), and optionally the dequantised bf16 values.
+__device__ __forceinline__ uint32_t quant_lane(const uint32_t (&w)[8], float enc, const float* s_rcp,
+                                               uint32_t& lo, uint32_t& hi) {
+  const uint32_t s = block_scale_code(bf16x16_amax(w), enc);
+  const float r = s_rcp[s];
+  lo = bf16x8_codes(w, r);
+  hi = bf16x8_codes(w + 4, r);
+  if (!(r > 0.0f)) lo = hi = 0u;  // d == 0: every code of the block is 0
+  return s;
+}
+
 // V8: x (and y) rows start on 32-byte boundaries, so each lane's 16 values move in one
 // 256-bit access.
+// Task geometry: a warp task is 8 consecutive 64-value groups (512 columns) of one row;
+// tpr tasks per row. When tpr <= the number of warps, warp w keeps column chunk w % tpr
+// and walks rows w / tpr, + nwarps / tpr, ... (no division in the loop; the few warps past
+// (nwarps / tpr) * tpr idle); otherwise every warp walks all rows and column chunks w,
+// w + nwarps, ... Rows are walked from the last one up, two per iteration (two loads in
+// flight per lane).
 template <bool V8>
 __global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(const Quant2Args a) {
   using namespace q2cfg;
@@ -542,33 +577,48 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(con
 
   const uint64_t stream = l2_policy_evict_first();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane & 3;                       // block of the lane's 64-value group
-  const int64_t ng = a.cols >> 6;                 // 64-value groups (scale words) per row
-  const int64_t tpr = (ng + 7) >> 3;              // warp tasks per row: 8 groups each
+  const int sub = lane & 3;                        // block of the lane's 64-value group
+  const int64_t ng = a.cols >> 6;                  // 64-value groups (scale words) per row
+  const int64_t tpr = (ng + 7) >> 3;               // warp tasks per row
   const int64_t rows_pad = (a.rows + 127) & ~int64_t(127);
-  const int64_t tasks = rows_pad * tpr;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * QUANT_WARPS;
-  for (int64_t t = tasks - 1 - (static_cast<int64_t>(blockIdx.x) * QUANT_WARPS + warp); t >= 0; t -= nwarps) {
-    const int64_t row = t / tpr;
-    const int64_t g = (t - row * tpr) * 8 + (lane >> 2);
-    const bool live = g < ng && row < a.rows;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * QUANT_WARPS + warp;
+  int64_t c0, cstep, r0, rstep;
+  if (tpr <= nwarps) {
+    rstep = nwarps / tpr;
+    r0 = w / tpr;
+    c0 = w - r0 * tpr;
+    cstep = tpr;
+    if (r0 >= rstep) return;
+  } else {
+    c0 = w;
+    cstep = nwarps;
+    r0 = 0;
+    rstep = 1;
+  }
+  const int64_t half_rows = a.rows >> 1;
+  const int64_t code_pitch = a.cols >> 1;
+  const int64_t nkb = a.cols >> 4;
+
+  auto src_row = [&](int64_t row) -> int64_t {
+    return a.interleave ? ((row & 1) ? half_rows + (row >> 1) : (row >> 1)) : row;
+  };
+  // scale word of each 64-value group: byte `sub` from lane 4k + sub (0 for padding rows)
+  auto store_word = [&](int64_t row, int64_t g, uint32_t s) {
+    uint32_t word = s << (8 * sub);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if (a.codes != nullptr && sub == 0 && g < ng) {
+      *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(row, 4 * g, nkb)) = word;
+    }
+  };
+  auto finish = [&](int64_t row, int64_t g, const uint32_t (&wv)[8], bool live) {
     uint32_t s = 0u;
     if (live) {
-      const int64_t src = a.interleave ? ((row & 1) ? (a.rows >> 1) + (row >> 1) : (row >> 1)) : row;
-      uint32_t w[8];
-      ld_global_32b<V8>(a.x + src * a.ldx + g * 64 + sub * 16, stream, w);
-      s = block_scale_code(bf16x16_amax(w), enc);
-      const float r = s_rcp[s];
-      float v[16];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        v[2 * j] = bf16_lo(w[j]);
-        v[2 * j + 1] = bf16_hi(w[j]);
-      }
-      uint32_t lo = block_codes8(v, r), hi = block_codes8(v + 8, r);
-      if (!(r > 0.0f)) lo = hi = 0u;  // d == 0: every code of the block is 0
+      uint32_t lo, hi;
+      s = quant_lane(wv, enc, s_rcp, lo, hi);
       if (a.codes != nullptr) {
-        *reinterpret_cast<uint2*>(a.codes + row * (a.cols >> 1) + g * 32 + sub * 8) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(a.codes + row * code_pitch + g * 32 + sub * 8) = make_uint2(lo, hi);
       }
       if (a.y != nullptr) {
         uint32_t o[8];
@@ -576,12 +626,28 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(con
         st_global_32b<V8>(a.y + row * a.ldy + g * 64 + sub * 16, o);
       }
     }
-    // the scale word of each 64-value group: byte `sub` from lane 4k + sub (0 for padding rows)
-    uint32_t word = s << (8 * sub);
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if (a.codes != nullptr && sub == 0 && g < ng) {
-      *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(row, 4 * g, a.cols >> 4)) = word;
+    store_word(row, g, s);
+  };
+
+  for (int64_t gc = c0; gc < tpr; gc += cstep) {
+    const int64_t g = gc * 8 + (lane >> 2);
+    const bool gl = g < ng;
+    int64_t rr = r0;
+    for (; rr + rstep < rows_pad; rr += 2 * rstep) {
+      const int64_t row0 = rows_pad - 1 - rr, row1 = row0 - rstep;
+      const bool l0 = gl && row0 < a.rows, l1 = gl && row1 < a.rows;
+      uint32_t w0[8], w1[8];
+      if (l0) ld_global_32b<V8>(a.x + src_row(row0) * a.ldx + g * 64 + sub * 16, stream, w0);
+      if (l1) ld_global_32b<V8>(a.x + src_row(row1) * a.ldx + g * 64 + sub * 16, stream, w1);
+      finish(row0, g, w0, l0);
+      finish(row1, g, w1, l1);
+    }
+    if (rr < rows_pad) {
+      const int64_t row0 = rows_pad - 1 - rr;
+      const bool l0 = gl && row0 < a.rows;
+      uint32_t w0[8];
+      if (l0) ld_global_32b<V8>(a.x + src_row(row0) * a.ldx + g * 64 + sub * 16, stream, w0);
+      finish(row0, g, w0, l0);
     }
   }
 }

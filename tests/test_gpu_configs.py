@@ -17,7 +17,7 @@ import torch
 import epilogues_nvfp4_quantize_b200 as ep
 from oracle import nvfp4_oracle as o
 import workloads as wk
-from gpu_util import assert_close, assert_requant_point13, bf16_to_np, device, quantize_gpu, read_nvfp4
+from gpu_util import assert_close, assert_close_chain, assert_requant_point13, bf16_to_np, device, quantize_gpu, read_nvfp4
 
 pytestmark = pytest.mark.gpu
 
@@ -113,7 +113,7 @@ def test_ffn_block_1k_image_up_then_down():
     qh, sh, _ = o.requantize(h_ref, G)
     qb, sb, gb = _oracle_b(down.N, down.K, down.seed)
     ref = o.bf16_round(o.gemm(o.dequantize(qh, sh, G), o.dequantize(qb, sb, gb)))
-    assert_close(bf16_to_np(out[torch.from_numpy(rows).to(device())]), ref, "ffn_down")
+    assert_close_chain(bf16_to_np(out[torch.from_numpy(rows).to(device())]), ref, "ffn_down")
 
 
 @pytest.mark.parametrize("M", wk.SWEEP_M)

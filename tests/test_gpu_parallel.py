@@ -12,7 +12,7 @@ import epilogues_nvfp4_quantize_b200 as ep
 from epilogues_nvfp4_quantize_b200.parallel import TPLayer
 import workloads as wk
 from oracle import nvfp4_oracle as o
-from gpu_util import assert_close, device
+from gpu_util import assert_close, assert_close_chain, device
 
 pytestmark = pytest.mark.gpu
 
@@ -58,7 +58,7 @@ def test_tp_layer_world1_equals_the_unsharded_kernels(M, reduce):
     qh, sh, _ = o.requantize(h_o, np.float32(G_h))
     qd, sd, gd = o.quantized_operand(wdc)
     out_o = o.gemm(o.dequantize(qh, sh, np.float32(G_h)), o.dequantize(qd, sd, gd))
-    assert_close(out.cpu().numpy().astype(np.float64), out_o, "TPLayer FFN vs oracle")
+    assert_close_chain(out.cpu().numpy().astype(np.float64), out_o, "TPLayer FFN vs oracle")
 
 
 def test_tp_layer_bf16_partials_world1_matches_the_oracle():
@@ -78,7 +78,7 @@ def test_tp_layer_bf16_partials_world1_matches_the_oracle():
     qh, sh, _ = o.requantize(h_o, np.float32(G_h))
     qd, sd, gd = o.quantized_operand(wd.cpu())
     out_o = o.bf16_round(o.gemm(o.dequantize(qh, sh, np.float32(G_h)), o.dequantize(qd, sd, gd)))
-    assert_close(out.float().cpu().numpy().astype(np.float64), out_o, "TPLayer bf16 partials vs oracle")
+    assert_close_chain(out.float().cpu().numpy().astype(np.float64), out_o, "TPLayer bf16 partials vs oracle")
 
 
 def test_signal_barrier_passes_alone_and_times_out_into_a_status():
