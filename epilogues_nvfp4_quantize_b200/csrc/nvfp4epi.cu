@@ -35,7 +35,6 @@ struct DeviceInfo {
   bool gemm_attr_set[2 * kEpiKinds] = {};
   bool pair_attr_set[2 * kEpiKinds] = {};
   int pair_clusters[2 * kEpiKinds] = {};
-  bool quant_attr_set = false;
   int quant_ctas_per_sm[2] = {0, 0};  // resident CTAs of quantize_rows_kernel<V8 = false, true>
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -238,69 +237,6 @@ nvfp4_status run_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, void* D, int
 }
 
 }  // namespace
-
-// Launch of the streaming quantiser (quantize.cuh) for nvfp4_quantize and
-// nvfp4_fake_quantize: codes/sf and/or the dequantised bf16 y.
-static nvfp4_status launch_quantize_stream(DeviceInfo* info, const void* x, int64_t rows, int64_t cols,
-                                           int64_t ldx, int compute_amax, bool inter, float* gscale,
-                                           uint8_t* codes, uint8_t* sf, uint16_t* y, int64_t ldy, void* workspace,
-                                           cudaStream_t stream) {
-  // stage shape: G boxes of R rows x 64 columns, G * R = 512. Four boxes of 128 rows (from
-  // 256 columns up) issue a quarter of the TMA loads of sixteen 32-row boxes; measured on
-  // 16384 x 3072, the quantiser is 11% faster.
-  const int64_t num_g = cols / 64;
-  int G = 4;
-  while (G > 1 && G > num_g) G >>= 1;
-  const int R = G >= 2 ? 512 / G : 256;
-  CUtensorMap tmX;
-  if (!make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(cols),
-                   static_cast<uint64_t>(rows), static_cast<uint64_t>(ldx) * 2, 64,
-                   static_cast<uint32_t>(inter ? R / 2 : R), CU_TENSOR_MAP_SWIZZLE_128B))
-    return NVFP4_ERR_CUDA;
-  nvfp4::QuantArgs args{};
-  args.rows = rows;
-  args.cols = cols;
-  args.box_rows = R;
-  args.boxes = G;
-  args.interleave = inter ? 1 : 0;
-  args.compute_amax = compute_amax;
-  args.gscale = gscale;
-  args.codes = codes;
-  args.sf = sf;
-  args.y = y;
-  args.ldy = ldy;
-  args.wait_limit_ns = kWaitLimitNs;
-  if (compute_amax) {
-    args.amax_bits = static_cast<unsigned int*>(workspace);
-    args.arrived = args.amax_bits + 1;
-    if (cudaMemsetAsync(workspace, 0, 2 * sizeof(unsigned int), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
-  }
-  {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!info->quant_attr_set) {
-      if (cudaFuncSetAttribute(nvfp4::quantize_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               nvfp4::qcfg::SMEM_BYTES) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
-      info->quant_attr_set = true;
-    }
-  }
-  const int64_t rows_pad = (rows + 127) / 128 * 128;
-  const int64_t chunks = (rows_pad + R - 1) / R * ((num_g + G - 1) / G);
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;  // the amax pass ends in a grid barrier: all CTAs resident
-  attr[0].val.cooperative = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(chunks < info->sm_count ? chunks : info->sm_count), 1, 1);
-  cfg.blockDim = dim3(nvfp4::qcfg::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = nvfp4::qcfg::SMEM_BYTES;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, nvfp4::quantize_stream_kernel, tmX, args) != cudaSuccess) return NVFP4_ERR_CUDA;
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return launch_status();
-}
 
 // Launch of the two-kernel quantiser (quantize.cuh) for nvfp4_quantize and
 // nvfp4_fake_quantize: with compute_amax, the amax partials kernel then the quantise kernel

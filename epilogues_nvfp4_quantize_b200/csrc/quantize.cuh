@@ -1,7 +1,8 @@
 // nvfp4_quantize: bf16 -> NVFP4 (E2M1 codes, E4M3 block scales in the tensor-core scale
-// layout, FP32 per-tensor scale). HBM-bound. quantize_stream_kernel is the path of
-// nvfp4_quantize; quantize_kernel (one thread per 64 values, plain loads) serves the
-// allocation-free variant, whose amax reduction runs in kernels of its own.
+// layout, FP32 per-tensor scale). HBM-bound. amax_partial_kernel + quantize_rows_kernel are
+// the path of nvfp4_quantize and nvfp4_fake_quantize; quantize_kernel (one thread per 64
+// values, plain loads) serves the allocation-free variant, whose amax reduction runs in
+// kernels of its own.
 #pragma once
 
 #include "ptx.cuh"
@@ -55,43 +56,6 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
   *reinterpret_cast<uint32_t*>(sf + sf_word_offset(r, 4 * c, cols >> 4)) = word;
 }
 
-// =====================================================================================
-// Streaming quantiser: one persistent CTA per SM. A producer warp moves stages of
-// R rows x 64G columns of x (G boxes of R rows x 64 bf16, G x R = 512; G = 16 when x has at
-// least 1024 columns, so a stage reads 2 KB runs of 32 rows) into a shared-memory ring with
-// TMA. The 128-byte swizzle keeps the consumers' 16-byte reads free of bank conflicts. 16
-// consumer warps, one thread per (row, 64-column group), read them. With compute_amax the
-// CTAs first stream all of x for its amax (the loads ask L2 to keep x), meet at a bounded
-// grid barrier (cooperative launch: every CTA is resident), derive G = amax / (6 * 448),
-// then stream x again (from L2 where it stayed) and quantise.
-// =====================================================================================
-namespace qcfg {
-constexpr int CONSUMER_WARPS = 16;
-constexpr int CONSUMERS = CONSUMER_WARPS * 32;   // 512: 4 boxes x 128 rows
-constexpr int THREADS = CONSUMERS + 32;          // + TMA producer warp
-constexpr int STAGE_BYTES = CONSUMERS * 128;     // 64 KB: 512 units of 64 bf16
-constexpr int STAGES = 3;
-constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-constexpr int SMEM_BYTES = OFF_BAR + (2 * STAGES + 2) * 8 + 16 + 1024;  // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory");
-}  // namespace qcfg
-
-struct QuantArgs {
-  int64_t rows, cols;        // output rows (after the optional interleave) and columns
-  int box_rows;              // R: rows per stage (32 .. 256, a power of two)
-  int boxes;                 // G: 64-column boxes per stage (R * G <= 512)
-  int interleave;            // output row 2j <- input row j, 2j+1 <- input row rows/2 + j
-  int compute_amax;          // 1: derive G from amax(|x|); 0: use *gscale
-  unsigned int* amax_bits;   // workspace word 0 (zeroed by the caller's stream)
-  unsigned int* arrived;     // workspace word 1: grid-barrier counter (zeroed likewise)
-  float* gscale;
-  uint8_t* codes;            // codes and scales (or null: fake quantisation only)
-  uint8_t* sf;
-  uint16_t* y;               // quantise-dequantise output in bf16 (or null)
-  int64_t ldy;
-  uint64_t wait_limit_ns;
-};
-
 // Dequantised bf16 values of one 16-block: bf16(fp32(e2m1(q) * e4m3(s)) * G). The
 // level-scale products are exact in f16 (at most 2 + 4 significant bits, magnitudes from
 // 2^-10 to 2688), so they are formed two at a time with one f16x2 multiply.
@@ -118,273 +82,11 @@ __device__ __forceinline__ void dequant_block16_bf16(uint32_t c_lo, uint32_t c_h
   }
 }
 
-__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// All CTAs have arrived on *ctr (bounded wait; false on time-out).
-__device__ __forceinline__ bool grid_wait(const unsigned int* ctr, unsigned int target, uint64_t limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(ctr) < target) {
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-    __nanosleep(32);
-  }
-  return true;
-}
-
-// Largest magnitude of 64 bf16 values (32 packed words).
-__device__ __forceinline__ float bf16x64_amax(const uint4 (&v)[8]) {
-  uint32_t m = v[0].x;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-    for (int k = (q == 0 ? 1 : 0); k < 4; ++k) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[k]));
-  }
-  return fmaxf(fabsf(__uint_as_float(m << 16)), fabsf(__uint_as_float(m & 0xFFFF0000u)));
-}
-
-__global__ void __launch_bounds__(qcfg::THREADS, 1)
-    quantize_stream_kernel(const __grid_constant__ CUtensorMap tmX, const QuantArgs a) {
-  using namespace qcfg;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* empty = full + STAGES;
-  uint64_t* red_bar = empty + STAGES;  // every consumer warp has folded its amax into s_amax
-  uint64_t* go_bar = red_bar + 1;      // G is known (after the grid barrier)
-  unsigned int* s_amax = reinterpret_cast<unsigned int*>(go_bar + 1);
-  float* s_G = reinterpret_cast<float*>(s_amax + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(s_G + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint64_t limit = a.wait_limit_ns;
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < STAGES; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], CONSUMER_WARPS);
-    }
-    mbar_init(red_bar, CONSUMER_WARPS);
-    mbar_init(go_bar, 1);
-    *s_amax = 0u;
-    *s_G = 0.0f;
-    *abort_flag = 0;
-    fence_mbarrier_init();
-  }
-  __syncthreads();
-
-  const int R = a.box_rows, NB = a.boxes;
-  const int64_t num_g = a.cols >> 6;                       // 64-column groups
-  const int64_t rows_pad = (a.rows + 127) & ~int64_t(127);  // rows that carry scale words
-  const int64_t per_rs = (num_g + NB - 1) / NB;             // chunks per R-row slab
-  const int64_t chunks = ((rows_pad + R - 1) / R) * per_rs;
-  const int passes = a.compute_amax ? 2 : 1;
-  // This CTA's chunks are blockIdx.x + k * gridDim.x, k < my_chunks. The quantise pass after an
-  // amax pass walks them backwards: the chunks read last by the amax pass are the likeliest
-  // to still be in L2.
-  const int64_t my_chunks = blockIdx.x < chunks ? (chunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  auto chunk_of = [&](int pass, int64_t k) -> int64_t {
-    const int64_t kk = pass == 1 ? my_chunks - 1 - k : k;
-    return static_cast<int64_t>(blockIdx.x) + kk * gridDim.x;
-  };
-
-  if (warp == CONSUMER_WARPS) {
-    // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmX);
-      const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int pass = 0; ok && pass < passes; ++pass) {
-        const uint64_t pol = pass + 1 < passes ? keep : stream;
-        for (int64_t k = 0; k < my_chunks; ++k) {
-          const int64_t c = chunk_of(pass, k);
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, limit, 41)) {
-            ok = false;
-            break;
-          }
-          const int64_t rs = c / per_rs;
-          const int64_t g0 = (c - rs * per_rs) * NB;
-          const int nb = static_cast<int>(num_g - g0 < NB ? num_g - g0 : NB);
-          mbar_arrive_expect_tx(&full[stage], nb * R * 128);
-          uint8_t* sb = smem + stage * STAGE_BYTES;
-          for (int b = 0; b < nb; ++b) {
-            const int x = static_cast<int>((g0 + b) * 64);
-            if (!a.interleave) {
-              tma_load_2d_hint(sb + b * R * 128, &tmX, &full[stage], x, static_cast<int>(rs * R), pol);
-            } else {
-              // even output rows from the first half of x, odd ones from the second
-              tma_load_2d_hint(sb + b * R * 128, &tmX, &full[stage], x, static_cast<int>(rs * (R / 2)), pol);
-              tma_load_2d_hint(sb + b * R * 128 + (R / 2) * 128, &tmX, &full[stage], x,
-                               static_cast<int>((a.rows >> 1) + rs * (R / 2)), pol);
-            }
-          }
-          ++issued;
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        // give up: wait (bounded) for the loads this thread started, then leave
-        for (int i = 0; i < STAGES && i < issued; ++i) {
-          if (--stage < 0) {
-            stage = STAGES - 1;
-            phase ^= 1u;
-          }
-          (void)mbar_wait(&full[stage], phase, nullptr, limit, 41);
-        }
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------------ consumers
-  const int b = threadIdx.x / R;  // box of the stage (threads past R * NB stay idle)
-  const int i = threadIdx.x % R;  // row of the box
-  const int sr = a.interleave ? ((i & 1) ? R / 2 + (i >> 1) : (i >> 1)) : i;  // its row in shared memory
-  const uint32_t rowoff = static_cast<uint32_t>(b * R * 128 + sr * 128);
-  const int sw = sr & 7;  // 128-byte swizzle: 16-byte chunk q of the row sits at q ^ sw
-  int stage = 0;
-  uint32_t phase = 0;
-  float m = 0.0f, G = 0.0f, enc = 0.0f;
-  for (int pass = 0; pass < passes; ++pass) {
-    const bool quant = pass + 1 == passes;
-    if (quant) {
-      if (a.compute_amax) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) {
-          atomicMax(s_amax, __float_as_uint(m));
-          mbar_arrive(red_bar);
-        }
-        if (threadIdx.x == 0) {
-          bool good = mbar_wait(red_bar, 0, abort_flag, limit, 42);
-          if (good) {
-            if (*s_amax != 0u) atomicMax(a.amax_bits, *s_amax);
-            __threadfence();
-            atomicAdd(a.arrived, 1u);
-            good = grid_wait(a.arrived, gridDim.x, limit);
-            if (!good) {
-              *abort_flag = 1;
-              record_status(6, 43);
-            }
-          }
-          if (good) {
-            const float g = __fdiv_rn(__uint_as_float(ld_acquire_gpu(a.amax_bits)), kGlobalDiv);
-            *s_G = g;
-            if (blockIdx.x == 0) *a.gscale = g;
-          }
-          mbar_arrive(go_bar);
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(go_bar, 0, abort_flag, limit, 44)) || *abort_flag) return;
-        G = *s_G;
-      } else {
-        G = *a.gscale;
-      }
-      enc = scale_encode_factor(G);
-    }
-    for (int64_t k = 0; k < my_chunks; ++k) {
-      const int64_t c = chunk_of(pass, k);
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, limit, 45))) return;
-      const int64_t rs = c / per_rs;
-      const int64_t g = (c - rs * per_rs) * NB + b;
-      const int64_t r = rs * R + i;
-      if (b < NB && g < num_g && r < rows_pad) {
-        uint4 v[8];
-        if (r < a.rows) {
-          const uint8_t* src = smem + stage * STAGE_BYTES + rowoff;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) v[q] = *reinterpret_cast<const uint4*>(src + ((q ^ sw) << 4));
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) v[q] = make_uint4(0u, 0u, 0u, 0u);  // padding rows: zero scales
-        }
-        if (!quant) {
-          m = fmaxf(m, bf16x64_amax(v));
-        } else {
-          uint32_t cw[8];
-          uint32_t word = 0;
-#pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
-            const uint32_t w[8] = {v[2 * blk].x,     v[2 * blk].y,     v[2 * blk].z,     v[2 * blk].w,
-                                   v[2 * blk + 1].x, v[2 * blk + 1].y, v[2 * blk + 1].z, v[2 * blk + 1].w};
-            word |= quant_block16_bf16(w, G, enc, cw[2 * blk], cw[2 * blk + 1]) << (8 * blk);
-          }
-          if (a.codes != nullptr) {
-            // 32 bytes of codes per row: staged in the row's first two chunks of the stage,
-            // then stored as whole 32-byte sectors, lanes 2k and 2k+1 taking the halves of
-            // one row, 16 rows per instruction
-            uint8_t* mine = smem + stage * STAGE_BYTES + rowoff;
-            *reinterpret_cast<uint4*>(mine + ((0 ^ sw) << 4)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            *reinterpret_cast<uint4*>(mine + ((1 ^ sw) << 4)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-            __syncwarp();
-            const int i0 = i - lane;
-            const int hf = lane & 1;
-#pragma unroll
-            for (int rd = 0; rd < 2; ++rd) {
-              const int ii = i0 + 16 * rd + (lane >> 1);
-              const int sri = a.interleave ? ((ii & 1) ? R / 2 + (ii >> 1) : (ii >> 1)) : ii;
-              const int64_t rr = rs * R + ii;
-              if (rr < a.rows) {
-                const uint4 val = *reinterpret_cast<const uint4*>(smem + stage * STAGE_BYTES + b * R * 128 + sri * 128 +
-                                                                  ((hf ^ (sri & 7)) << 4));
-                *reinterpret_cast<uint4*>(a.codes + rr * (a.cols >> 1) + g * 32 + hf * 16) = val;
-              }
-            }
-            *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(r, 4 * g, a.cols >> 4)) = word;
-          }
-          if (a.y != nullptr) {
-            // The warp's 32 rows of y go back into its own rows of the stage (same swizzle),
-            // then leave as whole 128-byte lines: lanes 8k..8k+7 store the 8 chunks of one
-            // row, 4 rows per instruction.
-            __syncwarp();  // the code transposition above has read the stage rows
-            uint8_t* mine = smem + stage * STAGE_BYTES + rowoff;
-#pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
-              uint32_t o[8];
-              dequant_block16_bf16(cw[2 * blk], cw[2 * blk + 1], (word >> (8 * blk)) & 0xFFu, G, o);
-              *reinterpret_cast<uint4*>(mine + (((2 * blk) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-              *reinterpret_cast<uint4*>(mine + (((2 * blk + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-            }
-            __syncwarp();
-            const int i0 = i - lane;  // the warp's first row of the box
-            const int ch = lane & 7;
-#pragma unroll
-            for (int rd = 0; rd < 8; ++rd) {
-              const int ii = i0 + 4 * rd + (lane >> 3);
-              const int sri = a.interleave ? ((ii & 1) ? R / 2 + (ii >> 1) : (ii >> 1)) : ii;
-              const int64_t rr = rs * R + ii;
-              if (rr < a.rows) {
-                const uint4 val = *reinterpret_cast<const uint4*>(smem + stage * STAGE_BYTES + b * R * 128 + sri * 128 +
-                                                                  ((ch ^ (sri & 7)) << 4));
-                *reinterpret_cast<uint4*>(a.y + rr * a.ldy + g * 64 + ch * 8) = val;
-              }
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
-      if (++stage == STAGES) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-  }
-}
-
 // =====================================================================================
 // Two-kernel quantiser (the path of nvfp4_quantize and nvfp4_fake_quantize).
 //
 // 1. amax_partial_kernel streams x once (HBM-bound) and writes one partial max|x| per CTA
-//    into the caller's workspace. Its loads ask L2 to keep x.
+//    into the caller's workspace.
 // 2. quantize_rows_kernel is launched with programmatic dependent launch: its CTAs may
 //    become resident while the first kernel drains, and wait (griddepcontrol.wait) until
 //    that kernel's partials are visible. Each CTA reduces the partials to the tensor's amax,
@@ -464,7 +166,9 @@ __global__ void __launch_bounds__(q2cfg::AMAX_THREADS, CONTIG ? 2 : 1) amax_part
                                                                            float* __restrict__ partial) {
   __shared__ float s_red[32];
   griddep_launch_dependents();  // the quantise kernel waits for this grid's completion anyway
-  const uint64_t keep = l2_policy_evict_last();
+  // normal L2 priority: marking x evict-last was measured 2 us slower on 16384 x 3072 (the
+  // quantise kernel, walking the rows backwards, finds what stayed either way)
+  const uint64_t keep = l2_policy_evict_normal();
   const int64_t cpr = cols >> 4;  // 32-byte chunks per row
   const int64_t total = rows * cpr;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
