@@ -71,7 +71,7 @@ def workload_desc(M: int) -> str:
 # capture summarised in profiles/, keyed by a hash of the GEMM's device code: a value
 # taken on another version of the kernel is not reported.
 TRAFFIC_BY_SOURCE = {
-    "ece8ee9ea16ae6fa": 146.2e6,
+    "923de5902a1b1c2e": 146.2e6,
 }
 
 
@@ -977,6 +977,50 @@ def run_configs(args):
         raise SystemExit(f"device status {status}")
 
 
+def run_quantize_only(args):
+    """The activation quantiser alone on the step's x (M x 3072 bf16): back-to-back calls with
+    the amax pass and with a static scale, each call after a 256 MB buffer is written (so L2
+    starts with other data, as in the step), timed with CUDA events. One JSON line."""
+    import torch
+    import epilogues_nvfp4_quantize_b200 as ep
+    import workloads as wk
+    from epilogues_nvfp4_quantize_b200.build import build
+
+    build()
+    ep.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    M = args.M
+    x = wk.activations(M, K_IN, wk.outlier_count(K_IN), seed=0).to(dev)
+    xq = ep.NVFP4Tensor.empty(M, K_IN, dev)
+    ws = torch.empty(ep.quantize_workspace_bytes(), dtype=torch.uint8, device=dev)
+    scrub = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i, (e0, e1) in enumerate(evs):
+            scrub.fill_(i & 255)
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize(dev)
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
+
+    n = max(args.steps, 1)
+    for _ in range(args.warmup):
+        ep.nvfp4_quantize(x, xq, workspace=ws)
+    t_amax = timed(lambda: ep.nvfp4_quantize(x, xq, workspace=ws), n)
+    t_static = timed(lambda: ep.nvfp4_quantize(x, xq, compute_amax=False), n)
+    status = ep.read_device_status()
+    algo = M * K_IN * (2 + 0.5 + 1 / 16)
+    print(json.dumps({"quantize": f"{M}x{K_IN} bf16", "calls": n, "amax_us": round(t_amax, 2),
+                      "static_us": round(t_static, 2), "amax_gbs": round(algo / (t_amax * 1e-6) / 1e9, 1),
+                      "static_gbs": round(algo / (t_static * 1e-6) / 1e9, 1), "hbm_peak_gbs": peaks()["hbm_gbs"],
+                      "device_status": status}))
+    if status != 0:
+        raise SystemExit(f"device status {status}")
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -1029,6 +1073,8 @@ def main():
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--quantize-only", action="store_true",
+                    help="time the activation quantiser alone on the step's x (median of --steps calls)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -1038,6 +1084,8 @@ def main():
         run_sweep(args)
     elif args.configs:
         run_configs(args)
+    elif args.quantize_only:
+        run_quantize_only(args)
     else:
         run_cuda(args)
 
