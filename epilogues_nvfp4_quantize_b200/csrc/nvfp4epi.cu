@@ -35,7 +35,9 @@ struct DeviceInfo {
   bool gemm_attr_set[2 * kEpiKinds] = {};
   bool pair_attr_set[2 * kEpiKinds] = {};
   int pair_clusters[2 * kEpiKinds] = {};
-  int quant_ctas_per_sm[2] = {0, 0};  // resident CTAs of quantize_rows_kernel<V8 = false, true>
+  // resident CTAs of quantize_rows_kernel<V8 = false>, <V8 = true>, quantize_flat_kernel<Y =
+  // false>, <Y = true>
+  int quant_ctas_per_sm[4] = {0, 0, 0, 0};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -284,25 +286,33 @@ static nvfp4_status launch_quantize2(DeviceInfo* info, const void* x, int64_t ro
     qa.nparts = static_cast<int>(parts);
   }
   const bool v8 = x_v8 && y_v8;
+  // the flat kernel: x (and y) contiguous and 32-byte aligned, no interleave
+  const bool flat = v8 && !inter && ldx == cols && (y == nullptr || ldy == cols);
+  const int kind = flat ? (y != nullptr ? 3 : 2) : (v8 ? 1 : 0);
   {
     // CTAs that fit on an SM at once: the kernel's warps stride over the whole tensor, so a
     // grid larger than one wave would only queue CTAs behind it
     std::lock_guard<std::mutex> lock(g_mutex);
-    int& per_sm = info->quant_ctas_per_sm[v8 ? 1 : 0];
+    int& per_sm = info->quant_ctas_per_sm[kind];
     if (per_sm == 0) {
       int n = 0;
-      const cudaError_t e = v8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_rows_kernel<true>,
-                                                                               QUANT_THREADS, 0)
-                               : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_rows_kernel<false>,
-                                                                               QUANT_THREADS, 0);
+      const cudaError_t e =
+          kind == 3   ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_flat_kernel<true>,
+                                                                      QUANT_THREADS, 0)
+          : kind == 2 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_flat_kernel<false>,
+                                                                      QUANT_THREADS, 0)
+          : kind == 1
+              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_rows_kernel<true>, QUANT_THREADS, 0)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::quantize_rows_kernel<false>, QUANT_THREADS, 0);
       if (e != cudaSuccess || n < 1) return NVFP4_ERR_CUDA;
       per_sm = n;
     }
   }
   const int64_t rows_pad = (rows + 127) / 128 * 128;
-  const int64_t tasks = rows_pad * ((cols / 64 + 7) / 8);
+  // warp tasks: 128 blocks of 16 (flat), or 512 columns of one row (row kernel)
+  const int64_t tasks = flat ? (rows * (cols / 16) + 127) / 128 : rows_pad * ((cols / 64 + 7) / 8);
   int64_t grid = (tasks + QUANT_WARPS - 1) / QUANT_WARPS;
-  const int64_t full = static_cast<int64_t>(info->quant_ctas_per_sm[v8 ? 1 : 0]) * info->sm_count;
+  const int64_t full = static_cast<int64_t>(info->quant_ctas_per_sm[kind]) * info->sm_count;
   if (grid > full) grid = full;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
@@ -315,8 +325,10 @@ static nvfp4_status launch_quantize2(DeviceInfo* info, const void* x, int64_t ro
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = v8 ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<true>, qa)
-                           : cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<false>, qa);
+  const cudaError_t e = kind == 3   ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_flat_kernel<true>, qa)
+                        : kind == 2 ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_flat_kernel<false>, qa)
+                        : kind == 1 ? cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<true>, qa)
+                                    : cudaLaunchKernelEx(&cfg, nvfp4::quantize_rows_kernel<false>, qa);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();

@@ -252,12 +252,11 @@ __device__ __forceinline__ uint32_t quant_lane(const uint32_t (&w)[8], float enc
 // (nwarps / tpr) * tpr idle); otherwise every warp walks all rows and column chunks w,
 // w + nwarps, ... Rows are walked from the last one up, two per iteration (two loads in
 // flight per lane).
-template <bool V8>
-__global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(const Quant2Args a) {
-  using namespace q2cfg;
-  __shared__ float s_rcp[128];
-  __shared__ float s_red[32];
-  __shared__ float s_G;
+// Start of both quantise kernels: wait for the amax partials (or the producer of x), reduce
+// them to the tensor's amax and G = amax / (6 * 448) (or read the static G), and fill the
+// shared table of the reciprocal of every block scale d = e4m3(s) * G (0 where d is 0; code
+// 0x7F is NaN and never produced by the saturating conversion). Returns G.
+__device__ __forceinline__ float quant_setup(const Quant2Args& a, float* s_rcp, float* s_red, float* s_G) {
   griddep_wait();  // the amax partials (or the producer of x) are complete and visible
   if (a.partials != nullptr) {
     float m = 0.0f;
@@ -265,19 +264,27 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(con
     m = block_max(m, s_red);
     if (threadIdx.x == 0) {
       const float g = __fdiv_rn(m, kGlobalDiv);
-      s_G = g;
+      *s_G = g;
       if (blockIdx.x == 0) *a.gscale = g;
     }
   } else if (threadIdx.x == 0) {
-    s_G = *a.gscale;
+    *s_G = *a.gscale;
   }
   __syncthreads();
-  const float G = s_G;
-  const float enc = scale_encode_factor(G);
-  // reciprocal of every block scale d = e4m3(s) * G (0 where d is 0; code 0x7F is NaN and
-  // never produced by the saturating conversion)
+  const float G = *s_G;
   if (threadIdx.x < 128) s_rcp[threadIdx.x] = threadIdx.x == 0x7F ? 0.0f : block_inv_scale(threadIdx.x, G);
   __syncthreads();
+  return G;
+}
+
+template <bool V8>
+__global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(const Quant2Args a) {
+  using namespace q2cfg;
+  __shared__ float s_rcp[128];
+  __shared__ float s_red[32];
+  __shared__ float s_G;
+  const float G = quant_setup(a, s_rcp, s_red, &s_G);
+  const float enc = scale_encode_factor(G);
 
   const uint64_t stream = l2_policy_evict_first();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -352,6 +359,114 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS) quantize_rows_kernel(con
       uint32_t w0[8];
       if (l0) ld_global_32b<V8>(a.x + src_row(row0) * a.ldx + g * 64 + sub * 16, stream, w0);
       finish(row0, g, w0, l0);
+    }
+  }
+}
+
+// 4 x 4 byte transpose across the 4 lanes of a quad: lane m (m = lane & 3) holds bytes
+// M[m][0..3] in `v` and returns M[0..3][m]. Two exchanges: halfwords with lane m ^ 2 (byte
+// selectors sel_h: lanes 0-1 keep their low halfword and take the partner's low one, lanes
+// 2-3 keep their high halfword and take the partner's high one), then bytes with lane m ^ 1
+// (sel_b: even lanes keep bytes 0 and 2, odd lanes bytes 1 and 3).
+__device__ __forceinline__ uint32_t quad_transpose_bytes(uint32_t v, uint32_t sel_h, uint32_t sel_b) {
+  v = __byte_perm(v, __shfl_xor_sync(0xffffffffu, v, 2), sel_h);
+  return __byte_perm(v, __shfl_xor_sync(0xffffffffu, v, 1), sel_b);
+}
+
+// Flat form of quantize_rows_kernel, for a contiguous row-major x (ldx == cols) without the
+// interleave, x and y (if any, contiguous too) on 32-byte boundaries. x is then one sequence
+// of 16-value blocks, and block b's codes sit at byte 8 b of the code array. A warp task is
+// 128 consecutive blocks (4 KB of x, 32 scale words): lane i quantises blocks i, 32 + i,
+// 64 + i and 96 + i of it (coalesced 256-bit loads), then the lanes of each quad exchange
+// their scale bytes so that every lane stores one whole scale word. The row of a lane's
+// scale word is tracked incrementally, so the loop has no division. Tasks are walked from
+// the end of x, where the amax kernel read last.
+// When the amax kernel ran first (a plain launch, so x was complete before either kernel
+// started), the first task's loads are issued before the partials are reduced.
+// Y: the bf16 quantise-dequantise output y is written too (a.y is not read otherwise).
+template <bool Y>
+__global__ void __launch_bounds__(q2cfg::QUANT_THREADS, Y ? 3 : 4) quantize_flat_kernel(const Quant2Args a) {
+  using namespace q2cfg;
+  __shared__ float s_rcp[128];
+  __shared__ float s_red[32];
+  __shared__ float s_G;
+  const uint64_t stream = l2_policy_evict_first();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ng = a.cols >> 6;        // scale words per row
+  const int64_t words = a.rows * ng;     // scale words of the real rows
+  const int64_t nblocks = 4 * words;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * QUANT_WARPS;
+  int64_t t = ((nblocks + 127) >> 7) - 1 - (static_cast<int64_t>(blockIdx.x) * QUANT_WARPS + warp);
+  uint32_t w[4][8];
+  auto load_task = [&](int64_t task) {
+    const int64_t b0 = 128 * task + lane;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (b0 + 32 * k < nblocks) ld_global_32b<true>(a.x + (b0 + 32 * k) * 16, stream, w[k]);
+    }
+  };
+  const bool early = a.partials != nullptr;
+  if (early && t >= 0) load_task(t);
+  const float G = quant_setup(a, s_rcp, s_red, &s_G);
+  const float enc = scale_encode_factor(G);
+
+  const int m = lane & 3, q = lane >> 2;
+  const int64_t nkb = a.cols >> 4;       // 16-blocks per row
+  const int64_t rows_pad = (a.rows + 127) & ~int64_t(127);
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (a.codes != nullptr) {  // the scale words of the padding rows are 0
+    for (int64_t pw = words + tid; pw < rows_pad * ng; pw += nthreads) {
+      const int64_t row = pw / ng;
+      *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(row, 4 * (pw - row * ng), nkb)) = 0u;
+    }
+  }
+  if (t < 0) return;
+  if (!early) load_task(t);
+  // this lane's scale word: word 32 t + 8 m + q, i.e. group g of row `row` (32-bit: rows
+  // and groups per row are below 2^31); it is a real word while row < rows
+  const int64_t wd = 32 * t + 8 * m + q;
+  const int ngi = static_cast<int>(ng);
+  int row = static_cast<int>(wd / ng), g = static_cast<int>(wd - static_cast<int64_t>(row) * ng);
+  const int64_t wstep = 32 * nwarps;  // scale words per sweep of all warps
+  const int drow = static_cast<int>(wstep / ng), dg = static_cast<int>(wstep - drow * ng);
+  const int rows_i = static_cast<int>(a.rows);
+  const uint32_t sel_h = m < 2 ? 0x5410u : 0x3276u;
+  const uint32_t sel_b = (m & 1) ? 0x3715u : 0x6240u;
+  // this lane's first block of task t, and how many blocks from it on are real (only the
+  // first task walked, the last of x, can be partial)
+  int64_t b0 = 128 * t + lane;
+  int64_t rem = nblocks - b0;
+  const int64_t bstep = 128 * nwarps;  // blocks per sweep of all warps
+  for (bool first = true; t >= 0; t -= nwarps, b0 -= bstep, rem += bstep, first = false) {
+    if (!first) load_task(t);
+    uint32_t sw = 0u;  // byte k: scale of block b0 + 32 k
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t b = b0 + 32 * k;
+      if (32 * k < rem) {
+        uint32_t lo, hi;
+        const uint32_t s = quant_lane(w[k], enc, s_rcp, lo, hi);
+        sw |= s << (8 * k);
+        if (a.codes != nullptr) *reinterpret_cast<uint2*>(a.codes + b * 8) = make_uint2(lo, hi);
+        if constexpr (Y) {
+          uint32_t o[8];
+          dequant_block16_bf16(lo, hi, s, G, o);
+          st_global_32b<true>(a.y + b * 16, o);
+        }
+      }
+    }
+    // lane 4 q + m held byte m of the words of groups 8 k + q; now it holds the word of group
+    // 8 m + q (all four of its blocks are real when the word is)
+    sw = quad_transpose_bytes(sw, sel_h, sel_b);
+    if (a.codes != nullptr && row < rows_i) {
+      *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(row, 4 * g, nkb)) = sw;
+    }
+    g -= dg;
+    row -= drow;
+    if (g < 0) {
+      g += ngi;
+      --row;
     }
   }
 }

@@ -94,6 +94,22 @@ def test_quantize_strided_rows():
     _check_bitwise(big[:, 128:640].cpu().contiguous(), t)
 
 
+@pytest.mark.parametrize("rows,cols", [(256, 512), (130, 192)])
+def test_quantize_contiguous_off_a_32_byte_boundary(rows, cols):
+    """A contiguous x that starts 16 bytes past a 32-byte boundary takes the row kernel with
+    128-bit accesses; the same values at a 32-byte boundary take the flat kernel. Both match
+    the oracle bit for bit."""
+    x = wk.activations(rows, cols, 2, seed=rows)
+    flat = torch.empty(rows * cols + 8, dtype=torch.bfloat16, device=device())
+    view = flat[8:].view(rows, cols)
+    assert view.data_ptr() % 32 == 16
+    view.copy_(x.to(device()))
+    t = ep.NVFP4Tensor.empty(rows, cols, device())
+    ep.nvfp4_quantize(view, t)
+    _check_bitwise(x, t)
+    _check_bitwise(x, quantize_gpu(x))
+
+
 def test_quantize_reuses_workspace_across_calls():
     ws = torch.empty(ep.quantize_workspace_bytes(), dtype=torch.uint8, device=device())
     for seed in (1, 2):
