@@ -978,9 +978,10 @@ def run_configs(args):
 
 
 def run_quantize_only(args):
-    """The activation quantiser alone on the step's x (M x 3072 bf16): back-to-back calls with
-    the amax pass and with a static scale, each call after a 256 MB buffer is written (so L2
-    starts with other data, as in the step), timed with CUDA events. One JSON line."""
+    """The activation quantiser alone on the step's x (M x 3072 bf16), with the amax pass and
+    with a static scale, timed with CUDA events two ways: each call after a 256 MB buffer is
+    written (so L2 starts with other data, as in the step; median of `steps` calls), and
+    `steps` calls back to back with nothing in between (their mean). One JSON line."""
     import torch
     import epilogues_nvfp4_quantize_b200 as ep
     import workloads as wk
@@ -1006,17 +1007,33 @@ def run_quantize_only(args):
         torch.cuda.synchronize(dev)
         return statistics.median(e0.elapsed_time(e1) for e0, e1 in evs) * 1e3
 
+    def loop(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n * 1e3
+
     n = max(args.steps, 1)
     for _ in range(args.warmup):
         ep.nvfp4_quantize(x, xq, workspace=ws)
     t_amax = timed(lambda: ep.nvfp4_quantize(x, xq, workspace=ws), n)
     t_static = timed(lambda: ep.nvfp4_quantize(x, xq, compute_amax=False), n)
+    l_amax = loop(lambda: ep.nvfp4_quantize(x, xq, workspace=ws), n)
+    l_static = loop(lambda: ep.nvfp4_quantize(x, xq, compute_amax=False), n)
     status = ep.read_device_status()
     algo = M * K_IN * (2 + 0.5 + 1 / 16)
+
+    def gbs(t):
+        return round(algo / (t * 1e-6) / 1e9, 1)
+
     print(json.dumps({"quantize": f"{M}x{K_IN} bf16", "calls": n, "amax_us": round(t_amax, 2),
-                      "static_us": round(t_static, 2), "amax_gbs": round(algo / (t_amax * 1e-6) / 1e9, 1),
-                      "static_gbs": round(algo / (t_static * 1e-6) / 1e9, 1), "hbm_peak_gbs": peaks()["hbm_gbs"],
-                      "device_status": status}))
+                      "static_us": round(t_static, 2), "amax_gbs": gbs(t_amax), "static_gbs": gbs(t_static),
+                      "back_to_back": {"amax_us": round(l_amax, 2), "static_us": round(l_static, 2),
+                                       "amax_gbs": gbs(l_amax), "static_gbs": gbs(l_static)},
+                      "hbm_peak_gbs": peaks()["hbm_gbs"], "device_status": status}))
     if status != 0:
         raise SystemExit(f"device status {status}")
 
