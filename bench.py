@@ -980,8 +980,8 @@ def run_configs(args):
 def run_quantize_only(args):
     """The activation quantiser alone on the step's x (M x 3072 bf16), with the amax pass and
     with a static scale, timed with CUDA events two ways: each call after a 256 MB buffer is
-    written (so L2 starts with other data, as in the step; median of `steps` calls), and
-    `steps` calls back to back with nothing in between (their mean). One JSON line."""
+    written (so L2 starts with other data, as in the step; median of `steps` calls), and at
+    least 200 calls back to back with nothing in between (their mean). One JSON line."""
     import torch
     import epilogues_nvfp4_quantize_b200 as ep
     import workloads as wk
@@ -1021,8 +1021,9 @@ def run_quantize_only(args):
         ep.nvfp4_quantize(x, xq, workspace=ws)
     t_amax = timed(lambda: ep.nvfp4_quantize(x, xq, workspace=ws), n)
     t_static = timed(lambda: ep.nvfp4_quantize(x, xq, compute_amax=False), n)
-    l_amax = loop(lambda: ep.nvfp4_quantize(x, xq, workspace=ws), n)
-    l_static = loop(lambda: ep.nvfp4_quantize(x, xq, compute_amax=False), n)
+    n_loop = max(200, n)  # long enough for the back-to-back steady state
+    l_amax = loop(lambda: ep.nvfp4_quantize(x, xq, workspace=ws), n_loop)
+    l_static = loop(lambda: ep.nvfp4_quantize(x, xq, compute_amax=False), n_loop)
     status = ep.read_device_status()
     algo = M * K_IN * (2 + 0.5 + 1 / 16)
 
@@ -1031,7 +1032,7 @@ def run_quantize_only(args):
 
     print(json.dumps({"quantize": f"{M}x{K_IN} bf16", "calls": n, "amax_us": round(t_amax, 2),
                       "static_us": round(t_static, 2), "amax_gbs": gbs(t_amax), "static_gbs": gbs(t_static),
-                      "back_to_back": {"amax_us": round(l_amax, 2), "static_us": round(l_static, 2),
+                      "back_to_back": {"calls": n_loop, "amax_us": round(l_amax, 2), "static_us": round(l_static, 2),
                                        "amax_gbs": gbs(l_amax), "static_gbs": gbs(l_static)},
                       "hbm_peak_gbs": peaks()["hbm_gbs"], "device_status": status}))
     if status != 0:
