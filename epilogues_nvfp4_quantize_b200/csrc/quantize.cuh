@@ -390,7 +390,9 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS, Y ? 3 : 4) quantize_flat
   __shared__ float s_rcp[128];
   __shared__ float s_red[32];
   __shared__ float s_G;
-  const uint64_t stream = l2_policy_evict_first();
+  // x streams past L2 when only codes are written; with the bf16 output y, normal priority
+  // was measured faster (16384 x 3072 with amax: 46.8 against 50.3 us)
+  const uint64_t stream = Y ? l2_policy_evict_normal() : l2_policy_evict_first();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ng = a.cols >> 6;        // scale words per row
   const int64_t words = a.rows * ng;     // scale words of the real rows
