@@ -411,6 +411,13 @@ def run_cuda(args):
     for k in ("qkv_rmsnorm", "up_swiglu_requant", "down_plain"):
         kernels[k]["pct_fp4_datasheet"] = round(100.0 * kernels[k]["tflops"] / FP4_DATASHEET_TFLOPS, 2)
     kernels["quantize_x"]["pct_hbm"] = round(100.0 * kernels["quantize_x"]["gbs"] / pk["hbm_gbs"], 1)
+    # the same call alone, back to back: in the step it follows the FFN-down GEMM, whose
+    # dirty bf16 output in L2 is written back to HBM while x streams in
+    t_q = time_loop(lambda: ep.nvfp4_quantize(layer.x, layer.xq, workspace=layer.ws), 100, 5, torch)
+    q_gbs = (M * K_IN * 2 + M * K_IN * (0.5 + 1 / 16)) / (t_q * 1e-3) / 1e9
+    kernels["quantize_x"]["alone"] = {"us": round(t_q * 1e3, 2), "gbs": round(q_gbs, 1),
+                                      "pct_hbm": round(100.0 * q_gbs / pk["hbm_gbs"], 1),
+                                      "how": "100 calls back to back after the timed steps"}
 
     # ---- unfused comparison (separately timed, same step shapes)
     if not args.no_unfused:
