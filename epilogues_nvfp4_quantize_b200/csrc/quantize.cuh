@@ -425,14 +425,15 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS, Y ? 3 : 4) quantize_flat
   }
   if (t < 0) return;
   if (!early) load_task(t);
-  // this lane's scale word: word 32 t + 8 m + q, i.e. group g of row `row` (32-bit: rows
-  // and groups per row are below 2^31); it is a real word while row < rows
+  // this lane's scale word: word 32 t + 8 m + q, i.e. group g of row `row` (g in 32 bits:
+  // groups per row are below 2^25); it is a real word while row < rows
   const int64_t wd = 32 * t + 8 * m + q;
   const int ngi = static_cast<int>(ng);
-  int row = static_cast<int>(wd / ng), g = static_cast<int>(wd - static_cast<int64_t>(row) * ng);
+  int64_t row = wd / ng;
+  int g = static_cast<int>(wd - row * ng);
   const int64_t wstep = 32 * nwarps;  // scale words per sweep of all warps
-  const int drow = static_cast<int>(wstep / ng), dg = static_cast<int>(wstep - drow * ng);
-  const int rows_i = static_cast<int>(a.rows);
+  const int64_t drow = wstep / ng;
+  const int dg = static_cast<int>(wstep - drow * ng);
   const uint32_t sel_h = m < 2 ? 0x5410u : 0x3276u;
   const uint32_t sel_b = (m & 1) ? 0x3715u : 0x6240u;
   // this lane's first block of task t, and how many blocks from it on are real (only the
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS, Y ? 3 : 4) quantize_flat
     // lane 4 q + m held byte m of the words of groups 8 k + q; now it holds the word of group
     // 8 m + q (all four of its blocks are real when the word is)
     sw = quad_transpose_bytes(sw, sel_h, sel_b);
-    if (a.codes != nullptr && row < rows_i) {
+    if (a.codes != nullptr && row < a.rows) {
       *reinterpret_cast<uint32_t*>(a.sf + sf_word_offset(row, 4 * g, nkb)) = sw;
     }
     g -= dg;
