@@ -93,10 +93,11 @@ int64_t nvfp4_quantize_workspace_bytes(void);
  *                     entry ignored: every value the call reads it writes first). It holds
  *                     one partial amax per CTA of the first of two kernels; calls that
  *                     share a workspace must not overlap on the GPU. The first kernel reads
- *                     x once for its amax (asking L2 to keep it); the second, launched with
- *                     programmatic dependent launch, reduces the partials and quantises,
- *                     reading x again, mostly from L2. x rows that start on 32-byte
- *                     boundaries are read with 256-bit accesses.
+ *                     x once for its amax; the second, launched with programmatic dependent
+ *                     launch, reduces the partials and quantises, reading x again from its
+ *                     end, where the first kernel read last (that part is likeliest still in
+ *                     L2). x rows that start on 32-byte boundaries are read with 256-bit
+ *                     accesses.
  *   compute_amax = 0: *out.gscale is used as given (static scale, must be > 0 and finite);
  *                     workspace may be NULL.
  * Per block of 16, in IEEE float32: s = E4M3_rn_satfinite(amax_b * (1 / (6 G))) (s = 0
