@@ -1,6 +1,7 @@
 // nvfp4_quantize: bf16 -> NVFP4 (E2M1 codes, E4M3 block scales in the tensor-core scale
-// layout, FP32 per-tensor scale). HBM-bound. amax_partial_kernel + quantize_rows_kernel are
-// the path of nvfp4_quantize and nvfp4_fake_quantize; quantize_kernel (one thread per 64
+// layout, FP32 per-tensor scale). HBM-bound. amax_partial_kernel, then quantize_flat_kernel
+// (contiguous x) or quantize_rows_kernel (other layouts), are the path of nvfp4_quantize and
+// nvfp4_fake_quantize; quantize_kernel (one thread per 64
 // values, plain loads) serves the allocation-free variant, whose amax reduction runs in
 // kernels of its own.
 #pragma once
@@ -87,16 +88,17 @@ __device__ __forceinline__ void dequant_block16_bf16(uint32_t c_lo, uint32_t c_h
 //
 // 1. amax_partial_kernel streams x once (HBM-bound) and writes one partial max|x| per CTA
 //    into the caller's workspace.
-// 2. quantize_rows_kernel is launched with programmatic dependent launch: its CTAs may
+// 2. The quantise kernel is launched with programmatic dependent launch: its CTAs may
 //    become resident while the first kernel drains, and wait (griddepcontrol.wait) until
 //    that kernel's partials are visible. Each CTA reduces the partials to the tensor's amax,
 //    derives G = amax / (6 * 448), and fills a shared table of the 127 block-scale
-//    reciprocals 1 / (e4m3(s) * G). Then every lane quantises one 16-value block: one
-//    32-byte load (a warp reads 1 KB of a row), the block's E4M3 scale, one table lookup
-//    for the reciprocal, 16 products and 8 E2M1 conversions, an 8-byte code store; lanes
-//    4k..4k+3 are the 4 blocks of one scale word, assembled with two shuffles. Row tasks
-//    run in the reverse order of the first kernel's reads, so the data read last (likeliest
-//    still in L2) is quantised first.
+//    reciprocals 1 / (e4m3(s) * G). A lane quantises a 16-value block with one 32-byte
+//    load, the block's E4M3 scale, one table lookup for the reciprocal, 16 products and 8
+//    E2M1 conversions, and an 8-byte code store. quantize_flat_kernel gives each lane four
+//    blocks of a 128-block warp task and builds the scale words with a byte transpose
+//    within each quad; quantize_rows_kernel gives each lane one block of a 512-column row
+//    chunk and builds them with two shuffles. Both walk x in the reverse order of the first
+//    kernel's reads, so the data read last (likeliest still in L2) is quantised first.
 // No grid barrier and no workspace clearing: every partial a call reads is written by the
 // same call.
 // =====================================================================================
