@@ -476,6 +476,19 @@ __global__ void __launch_bounds__(q2cfg::QUANT_THREADS, Y ? 3 : 4) quantize_flat
   }
 }
 
+// (a0, a1) <- (a0 + b0, a1 + b1) and (b0, b1) <- (a0 - b0, a1 - b1): two butterflies with one
+// packed add and one packed subtract, each lane rounded like the scalar operation.
+__device__ __forceinline__ void butterfly_f32x2(float& a0, float& a1, float& b0, float& b1) {
+  asm("{\n\t.reg .b64 ra, rb, rs, rd;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 rs, ra, rb;\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rs;\n\t"
+      "mov.b64 {%2, %3}, rd;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
 // =====================================================================================
 // MXFP4 (OCP Microscaling: E2M1 elements, one E8M0 scale per 32) with an optional fixed
 // block-local transform, the 32-point Walsh-Hadamard matrix H_2 (x) ... (x) H_2 (page
@@ -511,16 +524,23 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
       }
     }
     if (hadamard) {
-      // fast Walsh-Hadamard transform, stage h maps (v[j], v[j+h]) to (a + b, a - b)
+      // fast Walsh-Hadamard transform, stage h maps (v[j], v[j+h]) to (a + b, a - b), stages
+      // h = 1, 2, 4, 8, 16 in that order. In the first four, the butterflies of j and j + 16
+      // have the same shape, so one packed add and one packed subtract (two IEEE float32
+      // operations each) do both; the last stage pairs j with j + 16 itself.
 #pragma unroll
-      for (int h = 1; h < 32; h <<= 1) {
+      for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           if (j & h) continue;
-          const float a = v[j], b = v[j + h];
-          v[j] = __fadd_rn(a, b);
-          v[j + h] = __fsub_rn(a, b);
+          butterfly_f32x2(v[j], v[j + 16], v[j + h], v[j + h + 16]);
         }
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float a = v[j], b = v[j + 16];
+        v[j] = __fadd_rn(a, b);
+        v[j + 16] = __fsub_rn(a, b);
       }
     }
     float amax = 0.0f;
