@@ -38,6 +38,7 @@ struct DeviceInfo {
   // resident CTAs of quantize_rows_kernel<V8 = false>, <V8 = true>, quantize_flat_kernel<Y =
   // false>, <Y = true>
   int quant_ctas_per_sm[4] = {0, 0, 0, 0};
+  int mx_ctas_per_sm[2] = {0, 0};  // resident CTAs of mx_quantize_kernel<V8 = false, true>
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -460,10 +461,33 @@ NVFP4_API nvfp4_status mxfp4_quantize(const void* x, int64_t rows, int64_t cols,
   const float g = (flags & MXFP4_HADAMARD32) ? 0.17677669529663689f : 1.0f;
   const int64_t rows_pad = (rows + 127) / 128 * 128;
   const int64_t threads = rows_pad * (cols / 32);
-  nvfp4::mx_quantize_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-      static_cast<const uint16_t*>(x), rows, cols, ldx, (flags & MXFP4_HADAMARD32) ? 1 : 0,
-      (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0,
-      static_cast<uint8_t*>(out.codes), static_cast<uint8_t*>(out.sf), out.gscale, g);
+  // 256-bit loads when every row of x starts on a 32-byte boundary; one wave of CTAs at the
+  // occupancy the runtime reports, walking the blocks with the grid's stride
+  const bool v8 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0 && (ldx % 16) == 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int& per_sm = info->mx_ctas_per_sm[v8 ? 1 : 0];
+    if (per_sm == 0) {
+      int n = 0;
+      const cudaError_t e = v8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::mx_quantize_kernel<true>, 256, 0)
+                               : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4::mx_quantize_kernel<false>, 256, 0);
+      if (e != cudaSuccess || n < 1) return NVFP4_ERR_CUDA;
+      per_sm = n;
+    }
+  }
+  int64_t grid = (threads + 255) / 256;
+  const int64_t full = static_cast<int64_t>(info->mx_ctas_per_sm[v8 ? 1 : 0]) * info->sm_count;
+  if (grid > full) grid = full;
+  const int had = (flags & MXFP4_HADAMARD32) ? 1 : 0, inter = (flags & NVFP4_SWIGLU_INTERLEAVE) ? 1 : 0;
+  if (v8) {
+    nvfp4::mx_quantize_kernel<true><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(x), rows, cols, ldx, had, inter, static_cast<uint8_t*>(out.codes),
+        static_cast<uint8_t*>(out.sf), out.gscale, g);
+  } else {
+    nvfp4::mx_quantize_kernel<false><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(x), rows, cols, ldx, had, inter, static_cast<uint8_t*>(out.codes),
+        static_cast<uint8_t*>(out.sf), out.gscale, g);
+  }
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return launch_status();
 }

@@ -497,31 +497,28 @@ __device__ __forceinline__ void butterfly_f32x2(float& a0, float& a1, float& b0,
 // 32 activations; the pages' transforms are learned, this one is fixed). One thread per
 // block of 32; lanes 4k..4k+3 hold the 4 blocks of one scale word.
 // =====================================================================================
-__global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                          int64_t cols, int64_t ldx, int hadamard, int interleave,
-                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                                          float* __restrict__ gscale, float g) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) *gscale = g;
-  const int64_t nb = cols >> 5;  // blocks of 32 per row (a multiple of 4)
-  const int64_t rows_pad = (rows + 127) & ~int64_t(127);
-  const int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const bool live = u < rows_pad * nb;
-  const int64_t r = live ? u / nb : 0, kb = live ? u - r * nb : 0;
+// One block of 32 of row r (block kb) for mx_quantize_kernel: its transform, E8M0 scale and
+// codes; the 4 lanes 4k..4k+3 of the calling warp assemble one scale word. Every lane of the
+// warp calls it (live = false for lanes past the padded rows).
+template <bool V8>
+__device__ __forceinline__ void mx_quantize_block(const uint16_t* __restrict__ x, int64_t rows, int64_t ldx,
+                                                  int hadamard, int interleave, uint8_t* __restrict__ codes,
+                                                  uint8_t* __restrict__ sf, int64_t nb, int64_t r, int64_t kb,
+                                                  bool live, int lane, uint64_t stream) {
+  const int64_t cols = nb << 5;
   float v[32];
   uint32_t e = 0;
   if (live && r < rows) {
     // with `interleave`, output row 2j reads input row j and 2j+1 reads input row rows/2 + j
     const int64_t src = interleave ? ((r & 1) ? (rows >> 1) + (r >> 1) : (r >> 1)) : r;
-    const uint4* p = reinterpret_cast<const uint4*>(x + src * ldx + kb * 32);
+    const uint16_t* p = x + src * ldx + kb * 32;
+    uint32_t w[16];
+    ld_global_32b<V8>(p, stream, *reinterpret_cast<uint32_t(*)[8]>(w));
+    ld_global_32b<V8>(p + 16, stream, *reinterpret_cast<uint32_t(*)[8]>(w + 8));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 q = __ldg(p + i);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[8 * i + 2 * k] = bf16_lo(w[k]);
-        v[8 * i + 2 * k + 1] = bf16_hi(w[k]);
-      }
+    for (int k = 0; k < 16; ++k) {
+      v[2 * k] = bf16_lo(w[k]);
+      v[2 * k + 1] = bf16_hi(w[k]);
     }
     if (hadamard) {
       // fast Walsh-Hadamard transform, stage h maps (v[j], v[j+h]) to (a + b, a - b), stages
@@ -564,11 +561,40 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
     *reinterpret_cast<uint4*>(codes + r * (cols >> 1) + kb * 16) = make_uint4(c[0], c[1], c[2], c[3]);
   }
   // the 4 blocks of a scale word sit in lanes 4k..4k+3 (nb % 4 == 0 keeps them in one row)
-  const int lane = threadIdx.x & 31;
   uint32_t word = e << (8 * (lane & 3));
   word |= __shfl_xor_sync(0xffffffffu, word, 1);
   word |= __shfl_xor_sync(0xffffffffu, word, 2);
   if (live && (lane & 3) == 0) *reinterpret_cast<uint32_t*>(sf + sf_word_offset(r, kb, nb)) = word;
+}
+
+template <bool V8>
+__global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                          int64_t cols, int64_t ldx, int hadamard, int interleave,
+                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+                                                          float* __restrict__ gscale, float g) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *gscale = g;
+  const uint64_t stream = l2_policy_evict_first();
+  const int64_t nb = cols >> 5;  // blocks of 32 per row (a multiple of 4)
+  const int64_t rows_pad = (rows + 127) & ~int64_t(127);
+  const int64_t total = rows_pad * nb;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  // One wave of threads walks the blocks with a stride of the whole grid (a multiple of 32,
+  // so the 4 lanes of a scale word stay in one warp); each thread's (row, block) advances
+  // by the stride's quotient and remainder, without a division in the loop.
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  int64_t r = u0 / nb, kb = u0 - (u0 / nb) * nb;
+  const int64_t drow = nthreads / nb, dkb = nthreads - drow * nb;
+  for (int64_t base = u0 - lane; base < total; base += nthreads) {
+    const bool live = base + lane < total;
+    mx_quantize_block<V8>(x, rows, ldx, hadamard, interleave, codes, sf, nb, r, kb, live, lane, stream);
+    kb += dkb;
+    r += drow;
+    if (kb >= nb) {
+      kb -= nb;
+      ++r;
+    }
+  }
 }
 
 }  // namespace nvfp4

@@ -42,6 +42,27 @@ def test_mx_quantize_matches_oracle_bitwise(rows, cols, hadamard):
     assert g == (float(np.float32(1 / np.sqrt(32))) if hadamard else 1.0)
 
 
+@pytest.mark.parametrize("hadamard", [False, True])
+def test_mx_quantize_off_a_32_byte_boundary_and_strided(hadamard):
+    """x starting 16 bytes past a 32-byte boundary (128-bit loads) and x with a row pitch
+    above cols: the same codes and scales as the oracle."""
+    rows, cols = 260, 512
+    x = wk.activations(rows, cols, 3, seed=17)
+    flat = torch.empty(rows * cols + 8, dtype=torch.bfloat16, device=device())
+    xo = flat[8:].view(rows, cols)
+    assert xo.data_ptr() % 32 == 16
+    xo.copy_(x.to(device()))
+    big = torch.zeros(rows, cols + 136, dtype=torch.bfloat16, device=device())
+    xs = big[:, 8:8 + cols]
+    xs.copy_(x.to(device()))
+    q_ref, e_ref = o.mx_quantize(o.hadamard32_fp32_order(x.float().numpy()) if hadamard else x.float().numpy())
+    for xin in (xo, xs):
+        t = ep.mxfp4_quantize(xin, ep.NVFP4Tensor.empty_mx(rows, cols, device()), hadamard=hadamard)
+        q, e, _, buf = _read_mx(t)
+        assert np.array_equal(e, e_ref) and np.array_equal(q, q_ref)
+        assert np.array_equal(buf, o.mx_pack_scales(e_ref, cols))
+
+
 def _check_transform_plain(q, e, xf):
     """Codes and E8M0 scales of the transformed tensor against the plain definition
     mx_quantize(hadamard32(x)): a scale may differ only in a block whose amax is within
